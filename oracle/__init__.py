@@ -1,0 +1,35 @@
+"""CPU oracle for group-32 4-bit weight-only quantization and the dequantize-fused
+linear.
+
+TEST INFRASTRUCTURE ONLY. Nothing in the product path imports this package: only
+``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may use it. It is a plain, slow, obviously-correct NumPy restatement of what the
+source pages define, shares no code, table or constant generator with the CUDA
+library, and is itself pinned by the ``-m "not gpu"`` tests against hand-worked
+examples, closed forms, invariants and brute force.
+
+Functions whose parity has no independent pin say so in their docstring
+("parity unpinned"): only ``quantize_asym_minmax``, which exists to shape
+synthetic input data for the asymmetric variant.
+"""
+
+from .w4_oracle import (  # noqa: F401
+    FLOOR,
+    GROUP,
+    STATUS,
+    bf16_bits_to_f32,
+    check_linear,
+    dequantize,
+    dequantize_asym_gidx,
+    f32_to_bf16_bits,
+    linear,
+    linear_asym_gidx,
+    pack_nibbles,
+    payload_bytes,
+    quantize_asym_minmax,
+    quantize_rtn,
+    unpack_signed,
+    unpack_unsigned,
+    validate,
+    validate_asym,
+)
