@@ -1,0 +1,463 @@
+"""Benchmark of the W4A16 group-32 linear on B200.
+
+Headline workload (one step): the decode GEMV at M = 1 over the three 4096-hidden decoder
+projections (N, K) = (4096, 4096), (14336, 4096), (4096, 14336), with RTN group-32 signed
+int4 codes and fp32 scales quantized on the GPU from W ~ N(0, 0.02^2) and bf16 x ~ N(0, 1).
+Metric: weight GB/s = packed payload bytes (codes + 4 * scales, the LoopQ payload_bytes)
+per second. Four rotating copies of the weights (336 MB > 126 MB L2) make every step read
+weights last touched three steps earlier, so L2 cannot serve them.
+
+The timed steps run as CUDA graphs with a timing event before every launch, so each
+kernel's duration is measured on the launching stream over the whole timed region. The
+JSON line also carries the end-to-end number (public Python API, pinned host x in, y out
+every step), the roofline of the GEMV kernel, the oracle timed on the host cores, and a
+per-workload detail block (odd-width dequant, batched decode, prefill TFLOP/s, asymmetric
+act-order, quantize).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs an independent replica (no collective on the data path);
+value = units processed by all ranks / max-over-ranks time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "W4A16 group-32 linear: weight GB/s (% of HBM peak) decode; TFLOP/s prefill"
+UNIT = "GB/s"
+L2_BYTES = 126 * 1024 * 1024
+ROTATE = 4
+GRAPH_CHUNK = 1000  # steps per captured graph
+
+
+def payload(N, K):
+    return N * ((K + 1) // 2) + 4 * N * ((K + 31) // 32)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def recorded_traffic(kernel_file, summary):
+    """Per-launch DRAM traffic of the GEMV from the committed ncu summary, or None when the
+    kernel source changed after the counters were taken."""
+    try:
+        text = open(os.path.join(ROOT, "profiles", summary)).read()
+        src = open(os.path.join(ROOT, "weight_only_int4_04_b200", "csrc", kernel_file), "rb").read()
+    except OSError:
+        return None
+    m = re.search(r"bench-traffic: sha256=([0-9a-f]+) bytes_per_step_launch_mean=([0-9.e+]+)", text)
+    if not m or m.group(1) != hashlib.sha256(src).hexdigest()[:16]:
+        return None
+    return float(m.group(2))
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, uuid):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-i", uuid,
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle as it stands
+# ---------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(i.get("num_threads", 1)) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(frac_rows=8):
+    """One bounded sample of the decode workload for the oracle: 1/frac_rows of the rows of
+    each of the three shapes (all K). Returns (callable, payload bytes per call, text)."""
+    import oracle as O
+    cases = []
+    for N, K in workloads.DECODE_SHAPES:
+        c = workloads.decode_case(N, K)
+        n = N // frac_rows
+        q, s = O.quantize_rtn(c["W"][:n])
+        cases.append((c["x"], O.pack_nibbles(q), s, K))
+
+    def run():
+        for x, codes, s, K in cases:
+            O.linear(x, codes, s, K)
+    nbytes = sum(payload(N // frac_rows, K) for N, K in workloads.DECODE_SHAPES)
+    return run, nbytes, f"oracle linear (dequantize + fp64 matmul) at M=1 on 1/{frac_rows} of the rows of each decode shape"
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    run, nbytes, text = oracle_sample()
+    for _ in range(max(args.warmup, 0)):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    value = args.steps * nbytes / dt / 1e9
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode GEMV M=1, (N,K) in (4096,4096),(14336,4096),(4096,14336); sampled rows",
+                   "sample": text, "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": text},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-detail", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import weight_only_int4_04_b200 as w4  # fails loudly without the built library
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # -- workload: three decode shapes, quantized by the library, 4 rotating copies ------
+    shapes = workloads.DECODE_SHAPES
+    sets, xs, ys = [], [], []
+    for N, K in shapes:
+        c = workloads.decode_case(N, K)
+        W = torch.from_numpy(c["W"]).to(dev)
+        codes, scales = w4.quantize_rtn(W)
+        del W
+        sets.append([(codes.clone(), scales.clone()) for _ in range(ROTATE)])
+        xs.append(torch.from_numpy(c["x_bits"].view(np.int16)).to(dev).view(torch.bfloat16))
+        ys.append(torch.empty((1, N), dtype=torch.bfloat16, device=dev))
+    step_bytes = sum(payload(N, K) for N, K in shapes)
+    algo_bytes = [payload(N, K) + 2 * K + 2 * N for N, K in shapes]  # weights + x + y per launch
+
+    def step(i, evs=None):
+        r = i % ROTATE
+        for j, (N, K) in enumerate(shapes):
+            if evs is not None:
+                evs[j].record()
+            codes, scales = sets[j][r]
+            w4.linear(xs[j], codes, scales, K, out=ys[j])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # -- capture the timed steps (graphs of up to GRAPH_CHUNK steps, an event per launch) --
+    graphs, launch_events = [], []
+    side = torch.cuda.Stream()
+    done = 0
+    while done < args.steps:
+        n = min(GRAPH_CHUNK, args.steps - done)
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in shapes] for _ in range(n)]
+        tail = torch.cuda.Event(enable_timing=True, external=True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(n):
+                step(done + i, evs[i])
+            tail.record()
+        graphs.append(g)
+        launch_events.append((evs, tail))
+        done += n
+    torch.cuda.synchronize()
+    graphs[0].replay()  # first replay uploads the graph; not part of the timing
+    torch.cuda.synchronize()
+
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    time.sleep(0.2)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for g in graphs:
+        g.replay()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # per-launch kernel durations over the whole timed region
+    per_shape_ms = [0.0 for _ in shapes]
+    for evs, tail in launch_events:
+        for i in range(len(evs)):
+            for j in range(len(shapes)):
+                nxt = evs[i][j + 1] if j + 1 < len(shapes) else (evs[i + 1][0] if i + 1 < len(evs) else tail)
+                per_shape_ms[j] += evs[i][j].elapsed_time(nxt)
+    launches = args.steps * len(shapes)
+    kernel_ms = sum(per_shape_ms)
+    hbm_peak, tc_peak, tc_sus, peak_kind = peaks()
+    achieved = args.steps * sum(algo_bytes) / (kernel_ms * 1e-3) / 1e9
+    value = world * args.steps * step_bytes / (ms * 1e-3) / 1e9
+
+    # -- end to end through the public API: pinned x in, y out, every step --------------
+    e2e_steps = min(args.steps, 5000)
+    hx = [x.cpu().pin_memory() for x in xs]
+    hy = [torch.empty_like(y, device="cpu").pin_memory() for y in ys]
+    dx = [torch.empty_like(x) for x in xs]
+    h2d = sum(x.numel() * 2 for x in xs)
+    d2h = sum(y.numel() * 2 for y in ys)
+
+    def e2e_step(i):
+        r = i % ROTATE
+        for j, (N, K) in enumerate(shapes):
+            dx[j].copy_(hx[j], non_blocking=True)
+            codes, scales = sets[j][r]
+            w4.linear(dx[j], codes, scales, K, out=ys[j])
+            hy[j].copy_(ys[j], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * e2e_steps * step_bytes / (e2e_ms * 1e-3) / 1e9
+
+    detail = None
+    if rank == 0 and not args.no_detail:
+        detail = run_detail(w4, dev, hbm_peak, tc_peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        run, nbytes, text = oracle_sample()
+        run()
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            run()
+            reps += 1
+            if time.perf_counter() - t0 > 10.0:
+                break
+        dt = time.perf_counter() - t0
+        cpu = {"value": reps * nbytes / dt / 1e9, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": text + f"; {reps} repetitions in {dt:.1f} s on {os.cpu_count()} host CPUs"}
+
+    if world > 1:
+        dist.barrier()
+        for g in graphs:
+            del g
+        graphs.clear()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    frac = achieved / hbm_peak
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 x int4 -> fp32", "data": "synthetic",
+        "config": {"workload": "decode GEMV M=1: (N,K) = (4096,4096), (14336,4096), (4096,14336); "
+                               "RTN group-32 int4 + fp32 scales from W~N(0,0.02^2); x bf16 ~N(0,1); no bias",
+                   "l2": f"inputs larger than L2: {ROTATE} rotating weight copies, {ROTATE * step_bytes / 2**20:.0f} MiB",
+                   "timing": "CUDA graphs of <=1000 steps, CUDA events on the launching stream",
+                   "parallelism": f"replicas x{world}"},
+        "clocks": clocks,
+        "gpu_launches": launches,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps,
+                "note": "public Python API per step: pinned-host x -> device, 3 linears, y -> pinned host; "
+                        "weights resident in HBM"},
+        "roofline": {"bound": "hbm", "kernel": "gemv_kernel<1,false>", "achieved": achieved, "peak": hbm_peak,
+                     "unit": "GB/s", "frac": frac, "peak_kind": peak_kind,
+                     "traffic": recorded_traffic("k_gemv.cu", "gemv_decode_m1.md"),
+                     "algorithmic_bytes_per_step": sum(algo_bytes),
+                     "per_shape_gbs": {f"{N}x{K}": args.steps * b / (t * 1e-3) / 1e9
+                                       for (N, K), b, t in zip(shapes, algo_bytes, per_shape_ms)},
+                     "per_shape_us": {f"{N}x{K}": 1e3 * t / args.steps for (N, K), t in zip(shapes, per_shape_ms)}},
+        "cpu_baseline": cpu,
+        "detail": detail,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_detail(w4, dev, hbm_peak, tc_peak):
+    """Other workloads of the build, each timed with CUDA events per call and an L2 flush
+    (a 256 MiB write) between calls outside the timed events; median of the calls."""
+    import torch
+
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    out = {}
+
+    def bf16(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    # odd-width dequant check (4096, 4095) -> bf16
+    c = workloads.decode_case(*workloads.ODD_DEQUANT_SHAPE)
+    codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
+    N, K = workloads.ODD_DEQUANT_SHAPE
+    o = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    t = time_calls(lambda: w4.dequantize(codes, scales, K, torch.bfloat16, out=o), 20, flush)
+    nb = payload(N, K) + 2 * N * K
+    out["dequant_4096x4095_bf16"] = {"us": 1e3 * t, "gbs": nb / t / 1e6, "frac_hbm": nb / t / 1e6 / hbm_peak}
+
+    # quantize (14336, 4096)
+    N, K = workloads.BATCHED_SHAPE
+    c = workloads.decode_case(N, K, M=64, config=3, bias=True)
+    W = torch.from_numpy(c["W"]).to(dev)
+    t = time_calls(lambda: w4.quantize_rtn(W, status=torch.zeros(1, dtype=torch.int32, device=dev)), 10, flush)
+    nb = 4 * N * K + payload(N, K)
+    out["quantize_14336x4096"] = {"us": 1e3 * t, "gbs": nb / t / 1e6, "frac_hbm": nb / t / 1e6 / hbm_peak}
+
+    # batched decode M in {8, 16, 32, 64}
+    codes, scales = w4.quantize_rtn(W)
+    del W
+    bias = torch.from_numpy(c["bias"]).to(dev)
+    xall = bf16(c["x_bits"])
+    for M in workloads.BATCHED_M:
+        x = xall[:M].contiguous()
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        t = time_calls(lambda: w4.linear(x, codes, scales, K, bias=bias, out=y), 30, flush)
+        fl = 2.0 * M * N * K
+        out[f"batched_M{M}_14336x4096"] = {"us": 1e3 * t, "weight_gbs": payload(N, K) / t / 1e6,
+                                           "frac_hbm": payload(N, K) / t / 1e6 / hbm_peak,
+                                           "tflops": fl / t / 1e9}
+
+    # prefill GEMMs
+    for M, N, K in workloads.PREFILL_SHAPES:
+        c = workloads.decode_case(N, K, M=M, config=4)
+        codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
+        x = bf16(c["x_bits"])
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        t = time_calls(lambda: w4.linear(x, codes, scales, K, out=y), 5, flush)
+        fl = 2.0 * M * N * K
+        out[f"prefill_{M}x{N}x{K}"] = {"us": 1e3 * t, "tflops": fl / t / 1e9, "frac_tensor": fl / t / 1e9 / tc_peak}
+        del x, y, codes, scales
+
+    # asymmetric act-order, N=11008 K=4096 group 128
+    for M in workloads.ASYM_M:
+        a = workloads.asym_random_codes(M)
+        gi = torch.from_numpy(a["g_idx"]).to(dev)
+        sc, perm = w4.asym_prepare(torch.from_numpy(a["codes"]).to(dev), gi, a["K"], a["n_groups"])
+        s = torch.from_numpy(a["scales"]).to(dev)
+        z = torch.from_numpy(a["zeros"]).to(dev)
+        x = bf16(a["x_bits"])
+        b = torch.from_numpy(a["bias"]).to(dev)
+        y = torch.empty((M, a["N"]), dtype=torch.bfloat16, device=dev)
+        t = time_calls(lambda: w4.linear_asym_gidx(x, sc, s, z, gi, perm=perm, bias=b, out=y), 20, flush)
+        nb = a["codes"].size + 4 * a["scales"].size + a["zeros"].size + 4 * a["K"]
+        fl = 2.0 * M * a["N"] * a["K"]
+        out[f"asym_M{M}_11008x4096_g128"] = {"us": 1e3 * t, "weight_gbs": nb / t / 1e6,
+                                             "frac_hbm": nb / t / 1e6 / hbm_peak, "tflops": fl / t / 1e9}
+    return out
+
+
+def time_calls(fn, iters, flush):
+    import torch
+    ts = []
+    for _ in range(iters):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return float(np.median(ts))
+
+
+if __name__ == "__main__":
+    sys.exit(main())

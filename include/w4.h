@@ -1,0 +1,191 @@
+/*
+ * w4.h -- C ABI of the B200 (sm_100a) group-wise 4-bit weight-only library.
+ *
+ * The packed weight format is the LoopQ storage contract (page "loopq/packed_weight.py",
+ * class PackedLoopQWeight and its validate / _dequantize_validated / pack_weight):
+ *
+ *   W is [N, K]: N rows (output features), K columns (input features, "width").
+ *   codes  uint8  [N, ceil(K/2)], row-major, contiguous. Byte j of a row holds column 2j in
+ *          its LOW nibble and column 2j+1 in its HIGH nibble ("even_column_low"). For an odd K
+ *          the unused high nibble of the last byte is zero.
+ *   values signed two's-complement nibbles: a nibble v >= 8 stands for v - 16.
+ *          Format v1 forbids the nibble 8 (the narrow range [-7, 7]); v2 allows it (-8).
+ *   scales float32 [N, ceil(K/32)], row-major, finite and > 0: column k of row n is
+ *          dequantized as fp32(value * scales[n][k/32]); the last group covers only the
+ *          columns that exist.
+ *
+ * The asymmetric sub-channel variant (page "keras/src/layers/core/dense.py", int4 diff:
+ * _int4_build's kernel_scale / kernel_zero / g_idx and _int4_call's dequantize-with-zero)
+ * uses UNSIGNED nibbles u in [0, 15], a per-(row, group) zero point z (int8 holding [0, 15])
+ * and a column-to-group map g_idx: w[n][k] = fp32((u - z[n][g]) * s[n][g]) with g = g_idx[k].
+ * Scales and zeros are stored [N, n_groups] (rows = output features, as the packed codes).
+ *
+ * Conventions for every entry point:
+ *   - Every array pointer is DEVICE memory owned by the caller. The library keeps no pointer
+ *     after a call returns and allocates no device memory; scratch memory, where a call needs
+ *     it, comes in through (workspace, workspace_bytes).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). Calls that must read a result back (validation) synchronize that stream and
+ *     say so.
+ *   - Host-side checks (NULL pointers, sizes, dtype codes, alignment of the workspace) are
+ *     done before anything is enqueued and returned synchronously; nothing is enqueued on
+ *     an error.
+ *   - The hot calls (w4_dequantize, w4_linear, w4_linear_asym_gidx) do NOT check the content
+ *     of the codes and scales: the owner validates once before use (LoopQ's
+ *     _dequantize_validated fast path). w4_validate / w4_validate_asym do that check.
+ *   - Sizes are int64_t; N, K, M >= 1. K <= 2^24, N and M <= 2^31 - 1.
+ *   - A CUDA launch error is returned as W4_ERR_CUDA; w4_last_cuda_error() gives its code.
+ */
+#ifndef W4_H_
+#define W4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (no CUDA header is needed to include this file). */
+typedef struct CUstream_st *w4_stream_t;
+
+typedef enum {
+  W4_OK = 0,
+  W4_ERR_NULL = 1,          /* a required pointer is NULL                                  */
+  W4_ERR_SHAPE = 2,         /* a size is <= 0 or above its limit, or sizes do not agree    */
+  W4_ERR_DTYPE = 3,         /* unknown w4_dtype, or one the call does not offer            */
+  W4_ERR_NONFINITE = 4,     /* W holds NaN or +-Inf (pack_weight: "weight must be finite") */
+  W4_ERR_SCALE = 5,         /* a scale is not finite or not > 0 (validate)                 */
+  W4_ERR_HIGH_NIBBLE = 6,   /* odd K and a nonzero unused high nibble (validate)           */
+  W4_ERR_RESERVED_CODE = 7, /* format v1 and a nibble equal to 8 (validate)                */
+  W4_ERR_VERSION = 8,       /* format_version not in {1, 2} (validate)                     */
+  W4_ERR_GIDX = 9,          /* a g_idx entry outside [0, n_groups), or a bad perm          */
+  W4_ERR_ZERO = 10,         /* a zero point outside [0, 15]                                */
+  W4_ERR_UNSUPPORTED = 11,  /* a valid request this build does not serve                   */
+  W4_ERR_WORKSPACE = 12,    /* workspace too small or not 256-byte aligned                 */
+  W4_ERR_TIMEOUT = 13,      /* a bounded device-side wait expired (see w4_device_error)    */
+  W4_ERR_CUDA = 14          /* a CUDA runtime/driver call failed (see w4_last_cuda_error)  */
+} w4_status;
+
+typedef enum { W4_BF16 = 0, W4_F16 = 1, W4_F32 = 2, W4_F64 = 3 } w4_dtype;
+
+/*
+ * w4_quantize_rtn -- round-to-nearest symmetric group-32 quantization and packing.
+ * Page "loopq/packed_weight.py", pack_weight (checks and packing order); the rounding is
+ * round-half-to-even and the clip follows page "gemma/peft/_quantization_utils.py",
+ * uniform_quantize; the range is the narrow [-7, 7] that format v1 requires (validate).
+ * For each row n and group g (columns 32g .. min(32g+32, K)-1):
+ *     amax = max |W|;  s = max(fl32(amax / 7), 2^-126);  q = clamp(rne(fl32(W / s)), -7, 7)
+ *     scales[n][g] = s; codes packed as in the format above (odd K: high pad nibble = 0).
+ *   W        float32 [N, K] row-major, read only.
+ *   codes    out, uint8 [N, ceil(K/2)];  scales  out, float32 [N, ceil(K/32)].
+ *   d_status optional device int32: set to W4_ERR_NONFINITE if W holds NaN/Inf, left
+ *            unchanged otherwise (the caller zeroes it). If NULL, the call synchronizes
+ *            `stream` and returns W4_ERR_NONFINITE itself. Outputs are unspecified for a
+ *            non-finite W. The results are bit-identical to the definition above (IEEE
+ *            divide, no flush-to-zero).
+ */
+w4_status w4_quantize_rtn(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                          int32_t *d_status, w4_stream_t stream);
+
+/*
+ * w4_dequantize -- dense weight from the packed format.
+ * Page "loopq/packed_weight.py", _dequantize_validated: values * repeat_interleave(scales,
+ * 32)[:, :K] in fp32, then .to(output dtype): round-to-nearest-even to bf16/f16, exact
+ * widening to f64. Bit-identical to that definition.
+ *   format_version 1 or 2 (only checked for range here; content is not validated).
+ *   out  [N, K] row-major of `out_dtype` (W4_BF16, W4_F16, W4_F32 or W4_F64).
+ */
+w4_status w4_dequantize(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
+                        int format_version, w4_dtype out_dtype, void *out, w4_stream_t stream);
+
+/*
+ * w4_linear -- y = x . dequant(W)^T + bias, the dequantize-fused weight-only linear.
+ * Page "paddlenlp/quantization/quantization_linear.py", quant_weight_forward
+ * (weight_only_linear(x, weight, bias, weight_scale, weight_dtype, group_size)); page
+ * "keras/src/layers/core/dense.py", _int4_call (dequantize, matmul, add bias).
+ *   x     bf16 [M, K] row-major (activations are not quantized: weight-only, A16).
+ *   bias  optional fp32 [N] (NULL = none), added in fp32 before the final rounding.
+ *   y     out [M, N] row-major, W4_BF16 or W4_F32 (others: W4_ERR_DTYPE).
+ * Products and sums are formed in fp32 from the exact codes; where the tensor cores consume
+ * the weight, each weight enters as bf16(fp32(value * scale)). The result satisfies
+ *     |y - y_exact| <= 4e-3 * sum_k |x[m][k] * w[n][k]| + 1e-6 per element.
+ * The kernel is chosen by M (decode GEMV for small M, tensor-core GEMM for larger M) and
+ * by the alignment of the rows; every shape is served. workspace may be NULL when
+ * w4_linear_workspace_bytes(...) returns 0; otherwise it must hold that many bytes and be
+ * 256-byte aligned. Calls sharing one workspace must not overlap in time.
+ */
+w4_status w4_linear(const void *x, int64_t M, const uint8_t *codes, const float *scales,
+                    int64_t N, int64_t K, const float *bias, void *y, w4_dtype y_dtype,
+                    void *workspace, size_t workspace_bytes, w4_stream_t stream);
+
+/* Workspace bytes w4_linear needs for this shape (0 = none). */
+size_t w4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * w4_asym_prepare -- one-time act-order preparation of an asymmetric weight.
+ * Sorts the columns by group (stable: columns of one group keep their order) and writes
+ *   perm       out, int32 [K]: perm[j] = original column placed at sorted position j;
+ *   codes_out  out, uint8 [N, ceil(K/2)]: the unsigned nibbles reordered, column j of
+ *              codes_out = column perm[j] of codes_in (pad nibble zero).
+ * The result is the same weight with relabelled columns; w4_linear_asym_gidx given `perm`
+ * and `codes_out` gathers x through perm and reads each group's columns contiguously.
+ * g_idx entries outside [0, n_groups) give W4_ERR_GIDX (this call synchronizes `stream`).
+ */
+w4_status w4_asym_prepare(const uint8_t *codes_in, const int32_t *g_idx, int64_t N, int64_t K,
+                          int64_t n_groups, uint8_t *codes_out, int32_t *perm,
+                          w4_stream_t stream);
+
+/*
+ * w4_linear_asym_gidx -- y = x . dequant_asym(W)^T + bias with act-order g_idx.
+ * Page "keras/src/layers/core/dense.py", _int4_call sub-channel branch
+ * (dequantize_with_sz_map(kernel, kernel_scale, kernel_zero, g_idx), matmul, bias) and
+ * page "max/graph/quantization.py", QuantizationConfig (sym=False, desc_act=True).
+ *   codes    uint8 [N, ceil(K/2)] unsigned nibbles. If perm == NULL they are in original
+ *            column order; if perm != NULL they are the codes_out of w4_asym_prepare.
+ *   scales   float32 [N, n_groups]; zeros int8 [N, n_groups] in [0, 15];
+ *   g_idx    int32 [K]: group of ORIGINAL column k;  perm  int32 [K] or NULL.
+ *   x, bias, y, y_dtype, workspace: as w4_linear; the same tolerance holds.
+ */
+w4_status w4_linear_asym_gidx(const void *x, int64_t M, const uint8_t *codes,
+                              const float *scales, const int8_t *zeros, const int32_t *g_idx,
+                              const int32_t *perm, int64_t N, int64_t K, int64_t n_groups,
+                              const float *bias, void *y, w4_dtype y_dtype, void *workspace,
+                              size_t workspace_bytes, w4_stream_t stream);
+
+/*
+ * w4_validate -- the LoopQ content checks (page "loopq/packed_weight.py", validate) on a
+ * device-resident packed weight, reported in the page's order: W4_ERR_VERSION (format not
+ * 1 or 2), W4_ERR_SCALE, W4_ERR_HIGH_NIBBLE, W4_ERR_RESERVED_CODE (v1 only). Shape and
+ * dtype are the caller's contract. Synchronizes `stream`.
+ */
+w4_status w4_validate(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
+                      int format_version, w4_stream_t stream);
+
+/*
+ * w4_validate_asym -- checks for the asymmetric variant: W4_ERR_SCALE, W4_ERR_HIGH_NIBBLE
+ * (odd K), W4_ERR_ZERO (zero point outside [0, 15]), W4_ERR_GIDX (g_idx outside
+ * [0, n_groups)). Synchronizes `stream`.
+ */
+w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8_t *zeros,
+                           const int32_t *g_idx, int64_t N, int64_t K, int64_t n_groups,
+                           w4_stream_t stream);
+
+/* Error word written by bounded device-side waits (W4_OK if none expired). Reading it
+ * synchronizes the device and clears it. */
+w4_status w4_device_error(void);
+
+/* The cudaError_t of the last call that returned W4_ERR_CUDA (0 if none). */
+int w4_last_cuda_error(void);
+
+/* Static description of a status code. */
+const char *w4_status_string(w4_status status);
+
+/* Library ABI version (major * 100 + minor). */
+int w4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4_H_ */

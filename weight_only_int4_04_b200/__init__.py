@@ -1,0 +1,204 @@
+"""Python binding of libw4: group-wise 4-bit weight-only quantization and the
+dequantize-fused linear for one B200 (sm_100a).
+
+Argument marshalling only: every step runs in the CUDA kernels of ``libw4.so`` behind the
+C ABI in ``include/w4.h``. PyTorch provides device memory and the current stream. There is
+no CPU fallback: importing this package without the built library raises ImportError, and
+every call requires CUDA tensors.
+
+Packed format (page "loopq/packed_weight.py", PackedLoopQWeight): ``codes`` uint8
+``[N, ceil(K/2)]`` (even column in the low nibble, two's-complement nibbles) and ``scales``
+float32 ``[N, ceil(K/32)]``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw4.so")
+
+STATUS = {
+    0: "OK", 1: "NULL", 2: "SHAPE", 3: "DTYPE", 4: "NONFINITE", 5: "SCALE", 6: "HIGH_NIBBLE",
+    7: "RESERVED_CODE", 8: "VERSION", 9: "GIDX", 10: "ZERO", 11: "UNSUPPORTED", 12: "WORKSPACE",
+    13: "TIMEOUT", 14: "CUDA",
+}
+DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2, torch.float64: 3}
+
+EXPORTS = (
+    "w4_quantize_rtn", "w4_dequantize", "w4_linear", "w4_linear_workspace_bytes",
+    "w4_asym_prepare", "w4_linear_asym_gidx", "w4_validate", "w4_validate_asym",
+    "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
+)
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m weight_only_int4_04_b200.build` "
+        "(there is no CPU fallback)")
+
+_vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+lib = ctypes.CDLL(LIB_PATH)
+_SIGS = {
+    "w4_quantize_rtn": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
+    "w4_dequantize": [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp],
+    "w4_linear": [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _vp, _sz, _vp],
+    "w4_linear_workspace_bytes": [_i64, _i64, _i64],
+    "w4_asym_prepare": [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
+    "w4_linear_asym_gidx": [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp, _sz,
+                            _vp],
+    "w4_validate": [_vp, _vp, _i64, _i64, _i32, _vp],
+    "w4_validate_asym": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
+    "w4_device_error": [],
+    "w4_last_cuda_error": [],
+    "w4_status_string": [_i32],
+    "w4_version": [],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = ctypes.c_int
+lib.w4_linear_workspace_bytes.restype = ctypes.c_size_t
+lib.w4_status_string.restype = ctypes.c_char_p
+
+
+class W4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        msg = lib.w4_status_string(status).decode()
+        if self.name == "CUDA":
+            msg += f" (cudaError {lib.w4_last_cuda_error()})"
+        super().__init__(f"{where}: {self.name}: {msg}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise W4Error(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("w4: tensors must be contiguous CUDA tensors (no CPU fallback)")
+
+
+def quantize_rtn(W: torch.Tensor, status: torch.Tensor | None = None):
+    """RTN symmetric group-32 quantization of fp32 ``W [N, K]`` -> ``(codes, scales)``.
+
+    With ``status`` (an int32 CUDA tensor of one element, zeroed by the caller) the call
+    stays asynchronous and a non-finite W sets it to the NONFINITE code; without it the
+    call synchronizes and raises ``W4Error`` for a non-finite W."""
+    _need_cuda(W, status)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    N, K = W.shape
+    codes = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N, (K + 31) // 32), dtype=torch.float32, device=W.device)
+    _check(lib.w4_quantize_rtn(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(status), _stream()),
+           "w4_quantize_rtn")
+    return codes, scales
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, K: int, out_dtype=torch.float32,
+               format_version: int = 2, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Dense ``[N, K]`` weight of ``out_dtype`` (bf16, f16, f32 or f64)."""
+    _need_cuda(codes, scales, out)
+    N = codes.shape[0]
+    if out_dtype not in DTYPES:
+        raise ValueError("unsupported output dtype")
+    if out is None:
+        out = torch.empty((N, K), dtype=out_dtype, device=codes.device)
+    _check(lib.w4_dequantize(_ptr(codes), _ptr(scales), N, K, format_version, DTYPES[out_dtype], _ptr(out),
+                             _stream()), "w4_dequantize")
+    return out
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.w4_linear_workspace_bytes(M, N, K))
+
+
+def _workspace(M, N, K, device, workspace):
+    need = workspace_bytes(M, N, K)
+    if need == 0:
+        return None, 0
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def linear(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, K: int | None = None,
+           bias: torch.Tensor | None = None, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+           workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """``y = x . dequant(W)^T + bias`` for bf16 ``x [M, K]``; ``y [M, N]`` bf16 or fp32."""
+    _need_cuda(x, codes, scales, bias, out, workspace)
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    M, Kx = x.shape
+    K = Kx if K is None else K
+    if K != Kx:
+        raise ValueError("x width does not match K")
+    N = codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    ws, wsb = _workspace(M, N, K, x.device, workspace)
+    _check(lib.w4_linear(_ptr(x), M, _ptr(codes), _ptr(scales), N, K, _ptr(bias), _ptr(out),
+                         DTYPES[out.dtype], _ptr(ws), wsb, _stream()), "w4_linear")
+    return out
+
+
+def asym_prepare(codes: torch.Tensor, g_idx: torch.Tensor, K: int, n_groups: int):
+    """Sort the act-order columns by group: returns ``(codes_sorted, perm)``."""
+    _need_cuda(codes, g_idx)
+    N = codes.shape[0]
+    out = torch.empty_like(codes)
+    perm = torch.empty(K, dtype=torch.int32, device=codes.device)
+    _check(lib.w4_asym_prepare(_ptr(codes), _ptr(g_idx), N, K, n_groups, _ptr(out), _ptr(perm), _stream()),
+           "w4_asym_prepare")
+    return out, perm
+
+
+def linear_asym_gidx(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                     g_idx: torch.Tensor, perm: torch.Tensor | None = None, bias: torch.Tensor | None = None,
+                     out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Asymmetric act-order linear. ``g_idx`` may be float32 as Keras stores it; it is cast
+    to int32 (exact below 2**24)."""
+    if g_idx.dtype != torch.int32:
+        g_idx = g_idx.to(torch.int32)
+    _need_cuda(x, codes, scales, zeros, g_idx, perm, bias, out, workspace)
+    M, K = x.shape
+    N, G = scales.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    ws, wsb = _workspace(M, N, K, x.device, workspace)
+    _check(lib.w4_linear_asym_gidx(_ptr(x), M, _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), _ptr(perm),
+                                   N, K, G, _ptr(bias), _ptr(out), DTYPES[out.dtype], _ptr(ws), wsb,
+                                   _stream()), "w4_linear_asym_gidx")
+    return out
+
+
+def validate(codes: torch.Tensor, scales: torch.Tensor, K: int, format_version: int = 2) -> str:
+    """LoopQ content checks on the device; returns the status name ("OK" if valid)."""
+    _need_cuda(codes, scales)
+    return STATUS[lib.w4_validate(_ptr(codes), _ptr(scales), codes.shape[0], K, format_version, _stream())]
+
+
+def validate_asym(codes, scales, zeros, g_idx, K: int) -> str:
+    _need_cuda(codes, scales, zeros, g_idx)
+    return STATUS[lib.w4_validate_asym(_ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), codes.shape[0], K,
+                                       scales.shape[1], _stream())]
+
+
+def device_error() -> str:
+    return STATUS[lib.w4_device_error()]

@@ -1,0 +1,251 @@
+// Tensor-core W4A16 GEMM for prefill-sized M on sm_100a (tcgen05 + TMA + TMEM):
+//   y[m][n] = sum_k x[m][k] * bf16(fp32(q[n][k] * s[n][k/32])) + b[n]
+//
+// Swap-AB formulation: the dequantized weight tile is the MMA's A operand (M_mma = 128 weight
+// rows) and the activation tile is B (N_mma = 256 activation rows), so D = W_tile . x_tile^T
+// is a 128 x 256 fp32 tile of y^T held in tensor memory. This puts the larger MMA dimension
+// on the activations and dequantizes each weight tile once per 256 activation rows.
+//
+// One CTA per (128-row weight tile, 256-row activation tile); 10 warps, specialised:
+//   warp 0     TMA producer: per 64-column K block, the x tile (256 x 64 bf16, 128-byte
+//              swizzle), the code tile (128 rows x 32 bytes) and the scale tile
+//              (128 rows x 4 groups) land on one mbarrier;
+//   warp 1     allocates 256 TMEM columns; one thread issues 4 tcgen05.mma (K = 16 each)
+//              per K block and commits the stage back to the producer;
+//   warps 2-9  dequantize: thread (row, half) turns 16 code bytes + 1 scale into 32 bf16
+//              weights with LOP3/PRMT and fp32x2 arithmetic and stores them in the
+//              swizzled canonical K-major layout the MMA reads; then, after the last MMA,
+//              the same warps move D out of TMEM (tcgen05.ld), add the bias in fp32, round
+//              to the output dtype and store y.
+// A 4-stage ring of shared-memory stages (54 KB each) overlaps loads, dequantization and
+// MMA. All waits are bounded (see w4_sync.cuh).
+#include <cuda.h>
+
+#include "w4_tc.cuh"
+
+namespace w4i {
+
+namespace {
+
+constexpr int BM_W = 128;  // weight rows per tile (MMA M)
+constexpr int BN_X = 256;  // activation rows per tile (MMA N)
+constexpr int BK = 64;     // K per stage: one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int kThreads = 320;
+constexpr int kDequantWarp0 = 2;
+
+constexpr int A_BYTES = BM_W * BK * 2;    // 16 KB
+constexpr int B_BYTES = BN_X * BK * 2;    // 32 KB
+constexpr int C_BYTES = BM_W * (BK / 2);  // 4 KB of codes
+constexpr int S_BYTES = BM_W * 4 * 4;     // 2 KB: 4 scale groups per row (two stages' worth)
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_S = OFF_C + STAGES * C_BYTES;
+constexpr int OFF_BAR = OFF_S + STAGES * S_BYTES;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + 1 KB alignment slack
+constexpr uint32_t TX_BYTES = B_BYTES + C_BYTES + S_BYTES;
+constexpr uint32_t TMEM_COLS = BN_X;
+
+struct TcParams {
+  const float *bias;
+  void *y;
+  int64_t M, N, K;
+  int y_dtype;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
+                   const __grid_constant__ CUtensorMap tmap_scales, const TcParams p, int32_t *err) {
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base (the 128-byte swizzle atoms must start on 1024-byte boundaries)
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint64_t *full_load = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint64_t *full_a = full_load + STAGES;
+  uint64_t *empty = full_a + STAGES;
+  uint64_t *acc_full = empty + STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BM_W;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * BN_X;
+  const int KB = static_cast<int>((p.K + BK - 1) / BK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_load[s], 1);
+      mbar_init(&full_a[s], 8);  // one arrive per dequant warp
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err)) break;
+        mbar_arrive_expect_tx(&full_load[s], TX_BYTES);
+        tma_load_2d(smem + OFF_B + s * B_BYTES, &tmap_x, kb * BK, static_cast<int32_t>(m0), &full_load[s]);
+        tma_load_2d(smem + OFF_C + s * C_BYTES, &tmap_codes, kb * (BK / 2), static_cast<int32_t>(n0),
+                    &full_load[s]);
+        tma_load_2d(smem + OFF_S + s * S_BYTES, &tmap_scales, 4 * (kb / 2), static_cast<int32_t>(n0),
+                    &full_load[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM_W, BN_X);
+      const uint32_t a_base = smem_u32(smem + OFF_A);
+      const uint32_t b_base = smem_u32(smem + OFF_B);
+      for (int kb = 0; kb < KB; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
+        mbar_wait(&full_a[s], ph, abort_flag, err);
+        mbar_wait(&full_load[s], ph, abort_flag, err);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = umma_desc_sw128(a_base + s * A_BYTES + kk * 32);
+          const uint64_t bd = umma_desc_sw128(b_base + s * B_BYTES + kk * 32);
+          umma_bf16(tmem_d, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(acc_full);
+    }
+  } else {
+    // ---- dequantize into the A stages ----
+    const int q = warp & 3;                      // TMEM lane quarter this warp may access
+    const int half = (warp - kDequantWarp0) >> 2;  // which 32 of the stage's 64 columns
+    const int r = 32 * q + lane;                 // weight row inside the tile
+    const uint32_t a_row = smem_u32(smem + OFF_A) + r * 128;
+    for (int kb = 0; kb < KB; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
+      mbar_wait(&full_load[s], ph, abort_flag, err);
+      const uint4 cw = *reinterpret_cast<const uint4 *>(smem + OFF_C + s * C_BYTES + r * 32 + 16 * half);
+      const float sc = reinterpret_cast<const float *>(smem + OFF_S + s * S_BYTES)[r * 4 + (kb & 1) * 2 + half];
+      const uint64_t scale2 = (static_cast<uint64_t>(__float_as_uint(sc)) << 32) | __float_as_uint(sc);
+      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint4 v = dequant_word_bf16(words[t], scale2);
+        const uint32_t chunk = static_cast<uint32_t>(4 * half + t) ^ static_cast<uint32_t>(r & 7);
+        st_shared_v4(a_row + s * A_BYTES + chunk * 16, v);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full_a[s]);
+    }
+
+    // ---- epilogue: TMEM -> registers -> y ----
+    mbar_wait(acc_full, 0, abort_flag, err);
+    __syncwarp();  // tcgen05.ld is warp-collective; the lanes left the wait one by one
+    tc_fence_after();
+    const int64_t n = n0 + r;
+    const float b = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      const int col0 = 128 * half + 32 * c;
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(32 * q) << 16) + col0, v);
+      if (n < p.N) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int64_t m = m0 + col0 + j;
+          if (m < p.M) {
+            const float o = __uint_as_float(v[j]) + b;
+            if (p.y_dtype == W4_F32) {
+              static_cast<float *>(p.y)[m * p.N + n] = o;
+            } else {
+              static_cast<__nv_bfloat16 *>(p.y)[m * p.N + n] = __float2bfloat16_rn(o);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_d, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool gemm_tc_supports(const LinearParams &p) {
+  if (p.asym) return false;
+  const int64_t P = (p.K + 1) / 2, G = (p.K + 31) / 32;
+  if (p.K % 8 != 0 || P % 16 != 0 || G % 4 != 0) return false;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.codes) |
+                      reinterpret_cast<uintptr_t>(p.scales);
+  if (a % 16 != 0) return false;
+  if ((p.M + BN_X - 1) / BN_X > 65535 || (p.N + BM_W - 1) / BM_W > 0x7fffffffLL) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t stream) {
+  if (!gemm_tc_supports(p)) return cudaErrorNotSupported;
+  const int64_t P = (p.K + 1) / 2, G = (p.K + 31) / 32;
+  CUtensorMap mx, mc, ms;
+  if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, BK, BN_X,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.codes, P, p.N, P, BK / 2, BM_W, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.scales, G, p.N, G * 4, 4, BM_W,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  TcParams tp{p.bias, p.y, p.M, p.N, p.K, p.y_dtype};
+  const dim3 grid(static_cast<unsigned>((p.N + BM_W - 1) / BM_W), static_cast<unsigned>((p.M + BN_X - 1) / BN_X));
+  gemm_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(mx, mc, ms, tp, err);
+  return cudaGetLastError();
+}
+
+}  // namespace w4i

@@ -1,0 +1,297 @@
+// Standalone element-wise kernels: RTN quantize + pack, dequantize, content validation and
+// the act-order column reorder. All of them are HBM-bound streams: coalesced loads and
+// stores, no shared memory, grids sized in multiples of the SM count.
+#include <cfloat>
+
+#include "w4_internal.cuh"
+
+namespace w4i {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+int grid_for(int64_t work_items, int items_per_block) {
+  // Enough blocks to cover the work, capped at a multiple of 148 SMs x 8 resident blocks;
+  // the kernels are grid-stride loops.
+  int64_t blocks = (work_items + items_per_block - 1) / items_per_block;
+  const int64_t cap = 148LL * 8 * 4;
+  if (blocks > cap) blocks = cap;
+  return static_cast<int>(blocks < 1 ? 1 : blocks);
+}
+
+// ---------------------------------------------------------------------------
+// RTN quantize + pack (page "loopq/packed_weight.py", pack_weight; rounding and clip of
+// page "gemma/peft/_quantization_utils.py", uniform_quantize).
+// Eight lanes cooperate on one group of 32 columns, four columns per lane, so one warp
+// instruction reads four consecutive groups (512 contiguous bytes of W).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) quantize_rtn_kernel(const float *__restrict__ W,
+                                                                int64_t N, int64_t K,
+                                                                uint8_t *__restrict__ codes,
+                                                                float *__restrict__ scales,
+                                                                int32_t *__restrict__ status,
+                                                                int vec_ok) {
+  const int64_t G = (K + 31) / 32;
+  const int64_t P = (K + 1) / 2;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & 7;
+  const int64_t tasks = N * G;
+  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t warp_stride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  bool bad = false;
+  // A warp owns four consecutive tasks per trip; the trip count is warp-uniform so every
+  // lane reaches the shuffles below (lanes past the end work on zeros and store nothing).
+  for (int64_t wb = warp_id * 4; wb < tasks; wb += warp_stride * 4) {
+    const int64_t t = wb + (lane >> 3);
+    const bool active = t < tasks;
+    const int64_t n = active ? t / G : 0, g = active ? t % G : 0;
+    const int64_t c0 = 32 * g + 4 * sub;
+    const float *row = W + n * K;
+    float w[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (!active) {
+    } else if (vec_ok && c0 + 3 < K) {
+      const float4 v = __ldcs(reinterpret_cast<const float4 *>(row + c0));
+      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w[i] = (c0 + i < K) ? row[c0 + i] : 0.0f;
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      bad |= !isfinite(w[i]);
+      amax = fmaxf(amax, fabsf(w[i]));
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    // s = max(fl32(amax / 7), FLT_MIN): IEEE round-to-nearest divide.
+    const float s = fmaxf(__fdiv_rn(amax, 7.0f), FLT_MIN);
+    uint32_t nib[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int q = __float2int_rn(__fdiv_rn(w[i], s));  // round half to even
+      q = q < -7 ? -7 : (q > 7 ? 7 : q);
+      nib[i] = (c0 + i < K) ? (static_cast<uint32_t>(q) & 15u) : 0u;  // pad nibble = 0
+    }
+    const uint8_t b0 = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
+    const uint8_t b1 = static_cast<uint8_t>(nib[2] | (nib[3] << 4));
+    if (!active) continue;
+    uint8_t *crow = codes + n * P;
+    const int64_t j = c0 / 2;
+    if (j < P) crow[j] = b0;
+    if (j + 1 < P) crow[j + 1] = b1;
+    if (sub == 0) scales[n * G + g] = s;
+  }
+  if (bad) *status = W4_ERR_NONFINITE;
+}
+
+// ---------------------------------------------------------------------------
+// Dequantize (page "loopq/packed_weight.py", _dequantize_validated): fp32 value * scale,
+// then round-to-nearest-even into the output dtype (f64: exact widening).
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ T convert_out(float v);
+template <>
+__device__ __forceinline__ __nv_bfloat16 convert_out<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+template <>
+__device__ __forceinline__ __half convert_out<__half>(float v) {
+  return __float2half_rn(v);
+}
+template <>
+__device__ __forceinline__ float convert_out<float>(float v) {
+  return v;
+}
+template <>
+__device__ __forceinline__ double convert_out<double>(float v) {
+  return static_cast<double>(v);
+}
+
+__device__ __forceinline__ float signed_nibble(uint32_t byte, int hi) {
+  const int n = hi ? static_cast<int>(byte >> 4) : static_cast<int>(byte & 15u);
+  return static_cast<float>(n >= 8 ? n - 16 : n);
+}
+
+// Vector path: K % 8 == 0, so a row holds whole 4-byte code words and each word expands to
+// 8 consecutive outputs (16 bytes for bf16/f16). One thread per code word.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) dequant_vec_kernel(const uint8_t *__restrict__ codes,
+                                                               const float *__restrict__ scales,
+                                                               int64_t N, int64_t K,
+                                                               T *__restrict__ out) {
+  const int64_t words_per_row = K / 8;
+  const int64_t G = (K + 31) / 32;
+  const int64_t total = N * words_per_row;
+  const uint32_t *cw = reinterpret_cast<const uint32_t *>(codes);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / words_per_row, q = i % words_per_row;
+    const uint32_t w = __ldcs(cw + i);
+    const float s = __ldg(scales + n * G + q / 4);
+    __align__(16) T v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float val = signed_nibble((w >> (4 * e)) & 0xFFu, 0);
+      v[e] = convert_out<T>(__fmul_rn(val, s));
+    }
+    T *dst = out + n * K + q * 8;
+    constexpr int kVecs = (8 * sizeof(T)) / 16;
+#pragma unroll
+    for (int j = 0; j < kVecs; ++j) {
+      __stcs(reinterpret_cast<uint4 *>(dst) + j, reinterpret_cast<const uint4 *>(v)[j]);
+    }
+  }
+}
+
+// Generic path: any K (odd widths, partial groups, unaligned rows). One thread per code byte.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) dequant_generic_kernel(const uint8_t *__restrict__ codes,
+                                                                   const float *__restrict__ scales,
+                                                                   int64_t N, int64_t K,
+                                                                   T *__restrict__ out) {
+  const int64_t P = (K + 1) / 2;
+  const int64_t G = (K + 31) / 32;
+  const int64_t total = N * P;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / P, j = i % P;
+    const uint32_t b = codes[i];
+    const int64_t k0 = 2 * j;
+    const float s = scales[n * G + k0 / 32];
+    out[n * K + k0] = convert_out<T>(__fmul_rn(signed_nibble(b, 0), s));
+    if (k0 + 1 < K) out[n * K + k0 + 1] = convert_out<T>(__fmul_rn(signed_nibble(b, 1), s));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Content validation (page "loopq/packed_weight.py", validate; asymmetric extras).
+// Each thread ORs the rules it saw broken into a block-shared word; one atomic per block.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) validate_kernel(const uint8_t *__restrict__ codes,
+                                                            const float *__restrict__ scales,
+                                                            const int8_t *__restrict__ zeros,
+                                                            const int32_t *__restrict__ g_idx,
+                                                            int64_t N, int64_t K, int64_t n_scale_cols,
+                                                            int64_t n_groups, int check_v1,
+                                                            uint32_t *__restrict__ flags) {
+  __shared__ uint32_t block_flags;
+  if (threadIdx.x == 0) block_flags = 0;
+  __syncthreads();
+  uint32_t f = 0;
+  const int64_t P = (K + 1) / 2;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i = tid; i < N * n_scale_cols; i += step) {
+    const float s = scales[i];
+    if (!(isfinite(s) && s > 0.0f)) f |= FLAG_SCALE;
+    if (zeros != nullptr) {
+      const int z = zeros[i];
+      if (z < 0 || z > 15) f |= FLAG_ZERO;
+    }
+  }
+  if (check_v1) {
+    for (int64_t i = tid; i < N * P; i += step) {
+      const uint32_t b = codes[i];
+      if ((b & 15u) == 8u || (b >> 4) == 8u) f |= FLAG_RESERVED;
+    }
+  }
+  if (K & 1) {
+    for (int64_t n = tid; n < N; n += step) {
+      if (codes[n * P + P - 1] >> 4) f |= FLAG_HIGH_NIBBLE;
+    }
+  }
+  if (g_idx != nullptr) {
+    for (int64_t k = tid; k < K; k += step) {
+      const int32_t g = g_idx[k];
+      if (g < 0 || g >= n_groups) f |= FLAG_GIDX;
+    }
+  }
+  if (f) atomicOr(&block_flags, f);
+  __syncthreads();
+  if (threadIdx.x == 0 && block_flags) atomicOr(flags, block_flags);
+}
+
+// Column reorder for act-order weights: column j of the output is column perm[j] of the
+// input (unsigned nibbles), one thread per output byte; the pad nibble stays zero.
+__global__ void __launch_bounds__(kThreads) reorder_codes_kernel(const uint8_t *__restrict__ in,
+                                                                 const int32_t *__restrict__ perm,
+                                                                 int64_t N, int64_t K,
+                                                                 uint8_t *__restrict__ out) {
+  const int64_t P = (K + 1) / 2;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < N * P;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / P, j = i % P;
+    const uint8_t *row = in + n * P;
+    uint32_t v = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t col = 2 * j + h;
+      if (col < K) {
+        const int64_t src = perm[col];
+        const uint32_t b = row[src >> 1];
+        v |= ((src & 1) ? (b >> 4) : (b & 15u)) << (4 * h);
+      }
+    }
+    out[i] = static_cast<uint8_t>(v);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_rtn(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                                int32_t *status, cudaStream_t stream) {
+  const int64_t groups = N * ((K + 31) / 32);
+  const int vec_ok = (K % 4 == 0) && (reinterpret_cast<uintptr_t>(W) % 16 == 0);
+  quantize_rtn_kernel<<<grid_for(groups, kThreads / 8), kThreads, 0, stream>>>(W, N, K, codes, scales,
+                                                                              status, vec_ok);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t dequant_typed(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
+                                 void *out, cudaStream_t stream) {
+  T *o = static_cast<T *>(out);
+  const bool vec = (K % 8 == 0) && (reinterpret_cast<uintptr_t>(codes) % 4 == 0) &&
+                   (reinterpret_cast<uintptr_t>(out) % 16 == 0);
+  if (vec) {
+    dequant_vec_kernel<T><<<grid_for(N * (K / 8), kThreads), kThreads, 0, stream>>>(codes, scales, N, K, o);
+  } else {
+    dequant_generic_kernel<T><<<grid_for(N * ((K + 1) / 2), kThreads), kThreads, 0, stream>>>(codes, scales,
+                                                                                           N, K, o);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
+                              int out_dtype, void *out, cudaStream_t stream) {
+  switch (out_dtype) {
+    case W4_BF16: return dequant_typed<__nv_bfloat16>(codes, scales, N, K, out, stream);
+    case W4_F16: return dequant_typed<__half>(codes, scales, N, K, out, stream);
+    case W4_F32: return dequant_typed<float>(codes, scales, N, K, out, stream);
+    case W4_F64: return dequant_typed<double>(codes, scales, N, K, out, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_validate(const uint8_t *codes, const float *scales, const int8_t *zeros,
+                            const int32_t *g_idx, int64_t N, int64_t K, int64_t n_groups,
+                            int format_version, int asym, uint32_t *flags, cudaStream_t stream) {
+  const int64_t scale_cols = asym ? n_groups : (K + 31) / 32;
+  const int64_t work = N * ((K + 1) / 2);
+  validate_kernel<<<grid_for(work, kThreads * 4), kThreads, 0, stream>>>(
+      codes, scales, asym ? zeros : nullptr, asym ? g_idx : nullptr, N, K, scale_cols, n_groups,
+      (!asym && format_version == 1) ? 1 : 0, flags);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reorder_codes(const uint8_t *codes_in, const int32_t *perm, int64_t N, int64_t K,
+                                 uint8_t *codes_out, cudaStream_t stream) {
+  reorder_codes_kernel<<<grid_for(N * ((K + 1) / 2), kThreads), kThreads, 0, stream>>>(codes_in, perm, N,
+                                                                                      K, codes_out);
+  return cudaGetLastError();
+}
+
+}  // namespace w4i

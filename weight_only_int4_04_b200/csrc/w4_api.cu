@@ -1,0 +1,270 @@
+// C ABI entry points of libw4 (declared in include/w4.h): host-side argument checks, kernel
+// selection and error reporting. No device memory is allocated here; the only device state
+// is the static status words below (one per loaded library, shared by every call).
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
+#include "w4_internal.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+// Device words: validation flags and the non-finite flag of a quantize call that was given
+// no status pointer. Calls that use them synchronize, so they are never shared in flight.
+__device__ uint32_t g_validate_flags;
+__device__ int32_t g_quant_status;
+// Written by bounded device-side waits when they give up (read by w4_device_error).
+__device__ int32_t g_device_error;
+
+constexpr int64_t kMaxK = int64_t(1) << 24;
+constexpr int64_t kMaxRows = 0x7fffffffLL;
+
+w4_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return W4_ERR_CUDA;
+}
+
+bool sizes_ok(int64_t N, int64_t K) { return N >= 1 && K >= 1 && N <= kMaxRows && K <= kMaxK; }
+
+template <typename T>
+w4_status symbol_ptr(T **out, const T &sym) {
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, sym);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *out = static_cast<T *>(p);
+  return W4_OK;
+}
+
+w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspace_bytes,
+                     cudaStream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  int32_t *err = nullptr;
+  const w4_status st = symbol_ptr(&err, g_device_error);
+  if (st != W4_OK) return st;
+  // M dispatch: streaming GEMV for M = 1, the register GEMV for M <= 4, the tcgen05 GEMM
+  // above that; the generic kernel takes whatever the fast paths cannot (odd widths,
+  // unaligned rows, unsorted act-order maps).
+  cudaError_t e;
+  if (w4i::gemv_stream_supports(p)) {
+    e = w4i::launch_gemv_stream(p, err, stream);
+  } else if (w4i::gemv_supports(p)) {
+    e = w4i::launch_gemv(p, stream);
+  } else if (p.M > 4 && w4i::gemm_tc_supports(p)) {
+    e = w4i::launch_gemm_tc(p, err, stream);
+  } else {
+    e = w4i::launch_linear_generic(p, stream);
+  }
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int w4_version(void) { return 100; }
+
+int w4_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *w4_status_string(w4_status s) {
+  switch (s) {
+    case W4_OK: return "ok";
+    case W4_ERR_NULL: return "a required pointer is NULL";
+    case W4_ERR_SHAPE: return "size out of range or sizes do not agree";
+    case W4_ERR_DTYPE: return "unsupported dtype";
+    case W4_ERR_NONFINITE: return "weight must be finite";
+    case W4_ERR_SCALE: return "scales must be finite and positive";
+    case W4_ERR_HIGH_NIBBLE: return "nonzero unused high nibble";
+    case W4_ERR_RESERVED_CODE: return "reserved -8 code is outside the narrow signed range of format v1";
+    case W4_ERR_VERSION: return "unsupported packed-weight version";
+    case W4_ERR_GIDX: return "g_idx entry outside [0, n_groups)";
+    case W4_ERR_ZERO: return "zero point outside [0, 15]";
+    case W4_ERR_UNSUPPORTED: return "request not supported by this build";
+    case W4_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case W4_ERR_TIMEOUT: return "a bounded device-side wait expired";
+    case W4_ERR_CUDA: return "CUDA call failed";
+  }
+  return "unknown status";
+}
+
+w4_status w4_quantize_rtn(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                          int32_t *d_status, w4_stream_t stream) {
+  if (!W || !codes || !scales) return W4_ERR_NULL;
+  if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t *status = d_status;
+  if (!status) {
+    const w4_status st = symbol_ptr(&status, g_quant_status);
+    if (st != W4_OK) return st;
+    const cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  cudaError_t e = w4i::launch_quantize_rtn(W, N, K, codes, scales, status, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!d_status) {
+    int32_t host = 0;
+    e = cudaMemcpyAsync(&host, status, sizeof(host), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (host != 0) return W4_ERR_NONFINITE;
+  }
+  return W4_OK;
+}
+
+w4_status w4_dequantize(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
+                        int format_version, w4_dtype out_dtype, void *out, w4_stream_t stream) {
+  if (!codes || !scales || !out) return W4_ERR_NULL;
+  if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
+  if (format_version != 1 && format_version != 2) return W4_ERR_VERSION;
+  if (out_dtype != W4_BF16 && out_dtype != W4_F16 && out_dtype != W4_F32 && out_dtype != W4_F64)
+    return W4_ERR_DTYPE;
+  const cudaError_t e = w4i::launch_dequantize(codes, scales, N, K, out_dtype, out,
+                                               reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
+}
+
+size_t w4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)M;
+  (void)N;
+  (void)K;
+  return 0;
+}
+
+w4_status w4_linear(const void *x, int64_t M, const uint8_t *codes, const float *scales, int64_t N,
+                    int64_t K, const float *bias, void *y, w4_dtype y_dtype, void *workspace,
+                    size_t workspace_bytes, w4_stream_t stream) {
+  if (!x || !codes || !scales || !y) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || M < 1 || M > kMaxRows) return W4_ERR_SHAPE;
+  if (y_dtype != W4_BF16 && y_dtype != W4_F32) return W4_ERR_DTYPE;
+  const size_t need = w4_linear_workspace_bytes(M, N, K);
+  if (need > 0 && (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256))
+    return W4_ERR_WORKSPACE;
+  w4i::LinearParams p{};
+  p.x = static_cast<const __nv_bfloat16 *>(x);
+  p.codes = codes;
+  p.scales = scales;
+  p.bias = bias;
+  p.y = y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.y_dtype = y_dtype;
+  p.asym = 0;
+  return run_linear(p, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w4_status w4_asym_prepare(const uint8_t *codes_in, const int32_t *g_idx, int64_t N, int64_t K,
+                          int64_t n_groups, uint8_t *codes_out, int32_t *perm, w4_stream_t stream) {
+  if (!codes_in || !g_idx || !codes_out || !perm) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || n_groups < 1 || n_groups > K) return W4_ERR_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // One-time preparation: the stable sort of K column labels runs on the host.
+  std::vector<int32_t> gi(static_cast<size_t>(K));
+  cudaError_t e = cudaMemcpyAsync(gi.data(), g_idx, sizeof(int32_t) * K, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (int32_t g : gi)
+    if (g < 0 || g >= n_groups) return W4_ERR_GIDX;
+  std::vector<int32_t> order(static_cast<size_t>(K));
+  for (int64_t k = 0; k < K; ++k) order[k] = static_cast<int32_t>(k);
+  std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return gi[a] < gi[b]; });
+  e = cudaMemcpyAsync(perm, order.data(), sizeof(int32_t) * K, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = w4i::launch_reorder_codes(codes_in, perm, N, K, codes_out, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // `order` is host memory in flight
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
+}
+
+w4_status w4_linear_asym_gidx(const void *x, int64_t M, const uint8_t *codes, const float *scales,
+                              const int8_t *zeros, const int32_t *g_idx, const int32_t *perm,
+                              int64_t N, int64_t K, int64_t n_groups, const float *bias, void *y,
+                              w4_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                              w4_stream_t stream) {
+  if (!x || !codes || !scales || !zeros || !g_idx || !y) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || M < 1 || M > kMaxRows || n_groups < 1 || n_groups > K) return W4_ERR_SHAPE;
+  if (y_dtype != W4_BF16 && y_dtype != W4_F32) return W4_ERR_DTYPE;
+  const size_t need = w4_linear_workspace_bytes(M, N, K);
+  if (need > 0 && (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256))
+    return W4_ERR_WORKSPACE;
+  w4i::LinearParams p{};
+  p.x = static_cast<const __nv_bfloat16 *>(x);
+  p.codes = codes;
+  p.scales = scales;
+  p.zeros = zeros;
+  p.g_idx = g_idx;
+  p.perm = perm;
+  p.bias = bias;
+  p.y = y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_groups = static_cast<int>(n_groups);
+  p.y_dtype = y_dtype;
+  p.asym = 1;
+  return run_linear(p, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static w4_status run_validate(const uint8_t *codes, const float *scales, const int8_t *zeros,
+                              const int32_t *g_idx, int64_t N, int64_t K, int64_t n_groups,
+                              int format_version, int asym, cudaStream_t s, uint32_t *flags_out) {
+  uint32_t *flags = nullptr;
+  w4_status st = symbol_ptr(&flags, g_validate_flags);
+  if (st != W4_OK) return st;
+  cudaError_t e = cudaMemsetAsync(flags, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess)
+    e = w4i::launch_validate(codes, scales, zeros, g_idx, N, K, n_groups, format_version, asym, flags, s);
+  uint32_t host = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&host, flags, sizeof(host), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *flags_out = host;
+  return W4_OK;
+}
+
+w4_status w4_validate(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
+                      int format_version, w4_stream_t stream) {
+  if (!codes || !scales) return W4_ERR_NULL;
+  if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
+  if (format_version != 1 && format_version != 2) return W4_ERR_VERSION;
+  uint32_t f = 0;
+  const w4_status st = run_validate(codes, scales, nullptr, nullptr, N, K, 0, format_version, 0,
+                                    reinterpret_cast<cudaStream_t>(stream), &f);
+  if (st != W4_OK) return st;
+  if (f & w4i::FLAG_SCALE) return W4_ERR_SCALE;
+  if (f & w4i::FLAG_HIGH_NIBBLE) return W4_ERR_HIGH_NIBBLE;
+  if (f & w4i::FLAG_RESERVED) return W4_ERR_RESERVED_CODE;
+  return W4_OK;
+}
+
+w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8_t *zeros,
+                           const int32_t *g_idx, int64_t N, int64_t K, int64_t n_groups,
+                           w4_stream_t stream) {
+  if (!codes || !scales || !zeros || !g_idx) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || n_groups < 1 || n_groups > K) return W4_ERR_SHAPE;
+  uint32_t f = 0;
+  const w4_status st = run_validate(codes, scales, zeros, g_idx, N, K, n_groups, 2, 1,
+                                    reinterpret_cast<cudaStream_t>(stream), &f);
+  if (st != W4_OK) return st;
+  if (f & w4i::FLAG_SCALE) return W4_ERR_SCALE;
+  if (f & w4i::FLAG_HIGH_NIBBLE) return W4_ERR_HIGH_NIBBLE;
+  if (f & w4i::FLAG_ZERO) return W4_ERR_ZERO;
+  if (f & w4i::FLAG_GIDX) return W4_ERR_GIDX;
+  return W4_OK;
+}
+
+w4_status w4_device_error(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  int32_t host = 0;
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&host, g_device_error, sizeof(host));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (host != 0) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return static_cast<w4_status>(host);
+  }
+  return W4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,135 @@
+// Blackwell (sm_100a) tensor-core plumbing written as inline PTX: TMA tensor loads, the
+// tcgen05 MMA with its shared-memory and instruction descriptors, tensor-memory (TMEM)
+// allocation and loads, and the fences that order them.
+#pragma once
+
+#include <stdint.h>
+
+#include "w4_sync.cuh"
+
+namespace w4i {
+
+// 2-D TMA load of one box into shared memory, completing its bytes on `bar`. The innermost
+// coordinate `x` times the element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void *dst_smem, const void *tmap, int32_t x, int32_t y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand in the 128-byte swizzled canonical
+// layout: rows of 128 bytes (64 bf16), 8-row groups 1024 bytes apart, 16-byte chunks XORed
+// with the row index inside the group. Fields: start address >> 4 in bits [0,14), leading
+// byte offset >> 4 in [16,30) (unused by swizzled K-major; set to 1), stride byte offset
+// >> 4 in [32,46), the sm_100 descriptor version 1 in [46,48), swizzle mode 2 (128 B) in
+// [61,64). The tile must start on a 1024-byte boundary; a K step of 16 elements inside the
+// 128-byte row advances the start address by 32 bytes.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16: bf16 A and B (format 1 in bits [7,10)
+// and [10,13)), fp32 accumulator (format 1 in [4,6)), both operands K-major, N >> 3 in
+// [17,23), M >> 4 in [24,29).
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The mbarrier receives one arrive when every tcgen05 operation issued so far by this
+// thread has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Warp-wide TMEM allocation; the base address is written to shared memory at `slot`.
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Generic-proxy shared-memory writes become visible to the async proxy (tensor core, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp receives lane (base + i),
+// columns col .. col + 31. The warp may only address its own quarter of the 128 lanes.
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Eight signed nibbles of one code word (columns 8t .. 8t+7, even column low) -> eight
+// bf16 weights bf16(fp32(q * s)) in column order, packed as four bf16x2. Per column pair:
+// the nibble (xor 8) is placed in the low byte of the fp32 2^23 (PRMT), an exact fp32x2
+// subtract of 2^23 + 8 leaves q, one fp32x2 multiply by the scale rounds once, and the
+// pair is rounded to bf16 with round-to-nearest-even -- the same value w4_dequantize
+// produces for bf16 output.
+__device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, uint64_t scale2) {
+  const uint32_t lo = lop3_and_xor(w, 0x0F0F0F0Fu, 0x08080808u);       // even columns
+  const uint32_t hi = lop3_and_xor(w >> 4, 0x0F0F0F0Fu, 0x08080808u);  // odd columns
+  const uint64_t bias2 = 0xCB000008CB000008ull;                      // -(2^23 + 8), twice
+  uint32_t out[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t fe = prmt(lo, 0x00004B00u, 0x5440u | i);
+    const uint32_t fo = prmt(hi, 0x00004B00u, 0x5440u | i);
+    uint64_t v = (static_cast<uint64_t>(fo) << 32) | fe;
+    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(bias2));
+    asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(scale2));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+        : "=r"(out[i])
+        : "f"(__uint_as_float(static_cast<uint32_t>(v >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(v))));
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+}  // namespace w4i

@@ -121,3 +121,23 @@ def asym_case(M: int, N: int = ASYM_SHAPE[0], K: int = ASYM_SHAPE[1], group: int
     n_groups = (K + group - 1) // group
     return {"W": W, "x_bits": x_bits, "x": x, "bias": b, "g_idx": g_idx, "perm": perm,
             "n_groups": n_groups, "M": M, "N": N, "K": K, "group": group}
+
+
+def asym_random_codes(M: int, N: int = ASYM_SHAPE[0], K: int = ASYM_SHAPE[1], group: int = ASYM_GROUP,
+                      config: int = 5):
+    """Asymmetric inputs drawn directly as random storage (for timing only): packed bytes of
+    uniform unsigned nibbles (odd K: pad nibble zero), zero points uniform in [0, 15],
+    scales uniform in [1e-3, 4e-3], plus x, bias and an act-order map as in ``asym_case``."""
+    rng = rng_for(config, salt=1000 + M)
+    P = (K + 1) // 2
+    n_groups = (K + group - 1) // group
+    codes = rng.integers(0, 256, size=(N, P), dtype=np.uint8)
+    if K % 2:
+        codes[:, -1] &= 0x0F
+    zeros = rng.integers(0, 16, size=(N, n_groups)).astype(np.int8)
+    scales = rng.uniform(1e-3, 4e-3, size=(N, n_groups)).astype(np.float32)
+    x_bits, x = draw_x(rng, M, K)
+    b = draw_bias(rng, N)
+    g_idx, perm = draw_act_order(rng, K, group)
+    return {"codes": codes, "zeros": zeros, "scales": scales, "x_bits": x_bits, "x": x, "bias": b,
+            "g_idx": g_idx, "n_groups": n_groups, "M": M, "N": N, "K": K}
