@@ -7,8 +7,9 @@ Metric: weight GB/s = packed payload bytes (codes + 4 * scales, the LoopQ payloa
 per second. Four rotating copies of the weights (336 MB > 126 MB L2) make every step read
 weights last touched three steps earlier, so L2 cannot serve them.
 
-The timed steps run as CUDA graphs with a timing event before every launch, so each
-kernel's duration is measured on the launching stream over the whole timed region. The
+The timed steps run as CUDA graphs replayed back to back with CUDA events around the
+replays; every launch in the timed region is the GEMV, so its mean duration is the region
+time per launch (inter-launch gaps included). The
 JSON line also carries the end-to-end number (public Python API, pinned host x in, y out
 every step), the roofline of the GEMV kernel, the oracle timed on the host cores, and a
 per-workload detail block (odd-width dequant, batched decode, prefill TFLOP/s, asymmetric
@@ -179,6 +180,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-detail", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", default=None,
+                    help="time one named detail workload (e.g. prefill_4096x14336x4096) and exit")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -199,6 +202,13 @@ def main():
 
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
+    if args.only is not None:
+        hbm_peak, tc_peak, _, _ = peaks()
+        res = run_detail(w4, dev, hbm_peak, tc_peak, only=args.only, iters=args.steps, warmup=args.warmup)
+        if not res:
+            raise SystemExit(f"unknown workload {args.only}")
+        print(json.dumps({"only": args.only, **res[args.only]}), flush=True)
+        return 0
 
     # -- workload: three decode shapes, quantized by the library, 4 rotating copies ------
     shapes = workloads.DECODE_SHAPES
@@ -214,11 +224,9 @@ def main():
     step_bytes = sum(payload(N, K) for N, K in shapes)
     algo_bytes = [payload(N, K) + 2 * K + 2 * N for N, K in shapes]  # weights + x + y per launch
 
-    def step(i, evs=None):
+    def step(i):
         r = i % ROTATE
         for j, (N, K) in enumerate(shapes):
-            if evs is not None:
-                evs[j].record()
             codes, scales = sets[j][r]
             w4.linear(xs[j], codes, scales, K, out=ys[j])
 
@@ -226,21 +234,20 @@ def main():
         step(i)
     torch.cuda.synchronize()
 
-    # -- capture the timed steps (graphs of up to GRAPH_CHUNK steps, an event per launch) --
-    graphs, launch_events = [], []
+    # -- capture the timed steps as CUDA graphs of up to GRAPH_CHUNK steps. No event nodes
+    # inside the graphs: an event node between launches costs ~4-5 us of GPU time, more than
+    # a small GEMV itself, so the step is timed by events around the replays and the kernel
+    # time per launch is the timed region divided by the launches (all of them GEMVs).
+    graphs = []
     side = torch.cuda.Stream()
     done = 0
     while done < args.steps:
         n = min(GRAPH_CHUNK, args.steps - done)
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in shapes] for _ in range(n)]
-        tail = torch.cuda.Event(enable_timing=True, external=True)
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=side):
             for i in range(n):
-                step(done + i, evs[i])
-            tail.record()
+                step(done + i)
         graphs.append(g)
-        launch_events.append((evs, tail))
         done += n
     torch.cuda.synchronize()
     graphs[0].replay()  # first replay uploads the graph; not part of the timing
@@ -268,18 +275,31 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
 
-    # per-launch kernel durations over the whole timed region
-    per_shape_ms = [0.0 for _ in shapes]
-    for evs, tail in launch_events:
-        for i in range(len(evs)):
-            for j in range(len(shapes)):
-                nxt = evs[i][j + 1] if j + 1 < len(shapes) else (evs[i + 1][0] if i + 1 < len(evs) else tail)
-                per_shape_ms[j] += evs[i][j].elapsed_time(nxt)
     launches = args.steps * len(shapes)
-    kernel_ms = sum(per_shape_ms)
     hbm_peak, tc_peak, tc_sus, peak_kind = peaks()
-    achieved = args.steps * sum(algo_bytes) / (kernel_ms * 1e-3) / 1e9
+    # every launch of the timed region is the GEMV kernel: its average duration is the
+    # region time per launch (graph launch gaps included, so this is conservative)
+    achieved = args.steps * sum(algo_bytes) / (ms * 1e-3) / 1e9
     value = world * args.steps * step_bytes / (ms * 1e-3) / 1e9
+
+    # per-shape split, measured the same way on graphs of one shape (reported, not timed region)
+    per_shape_us = {}
+    for j, (N, K) in enumerate(shapes):
+        reps = 200
+        gj = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gj, stream=side):
+            for i in range(reps):
+                codes, scales = sets[j][i % ROTATE]
+                w4.linear(xs[j], codes, scales, K, out=ys[j])
+        gj.replay()
+        torch.cuda.synchronize()
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_ev.record(stream)
+        gj.replay()
+        b_ev.record(stream)
+        torch.cuda.synchronize()
+        per_shape_us[f"{N}x{K}"] = 1e3 * a_ev.elapsed_time(b_ev) / reps
+        del gj
 
     # -- end to end through the public API: pinned x in, y out, every step --------------
     e2e_steps = min(args.steps, 5000)
@@ -351,7 +371,7 @@ def main():
         "config": {"workload": "decode GEMV M=1: (N,K) = (4096,4096), (14336,4096), (4096,14336); "
                                "RTN group-32 int4 + fp32 scales from W~N(0,0.02^2); x bf16 ~N(0,1); no bias",
                    "l2": f"inputs larger than L2: {ROTATE} rotating weight copies, {ROTATE * step_bytes / 2**20:.0f} MiB",
-                   "timing": "CUDA graphs of <=1000 steps, CUDA events on the launching stream",
+                   "timing": "CUDA graphs of <=1000 steps replayed back to back, CUDA events on the launching stream around the replays",
                    "parallelism": f"replicas x{world}"},
         "clocks": clocks,
         "gpu_launches": launches,
@@ -359,13 +379,14 @@ def main():
                 "steps": e2e_steps,
                 "note": "public Python API per step: pinned-host x -> device, 3 linears, y -> pinned host; "
                         "weights resident in HBM"},
-        "roofline": {"bound": "hbm", "kernel": "gemv_kernel<1,false>", "achieved": achieved, "peak": hbm_peak,
+        "roofline": {"bound": "hbm", "kernel": "gemv_stream_kernel (M=1 decode GEMV)", "achieved": achieved, "peak": hbm_peak,
                      "unit": "GB/s", "frac": frac, "peak_kind": peak_kind,
                      "traffic": recorded_traffic("k_gemv.cu", "gemv_decode_m1.md"),
                      "algorithmic_bytes_per_step": sum(algo_bytes),
-                     "per_shape_gbs": {f"{N}x{K}": args.steps * b / (t * 1e-3) / 1e9
-                                       for (N, K), b, t in zip(shapes, algo_bytes, per_shape_ms)},
-                     "per_shape_us": {f"{N}x{K}": 1e3 * t / args.steps for (N, K), t in zip(shapes, per_shape_ms)}},
+                     "launch_us_mean": 1e3 * ms / launches,
+                     "per_shape_gbs": {f"{N}x{K}": b / us / 1e3
+                                       for (N, K), b, us in zip(shapes, algo_bytes, per_shape_us.values())},
+                     "per_shape_us": per_shape_us},
         "cpu_baseline": cpu,
         "detail": detail,
     }
@@ -373,74 +394,101 @@ def main():
     return 0
 
 
-def run_detail(w4, dev, hbm_peak, tc_peak):
-    """Other workloads of the build, each timed with CUDA events per call and an L2 flush
-    (a 256 MiB write) between calls outside the timed events; median of the calls."""
+def detail_workloads(w4, dev, hbm_peak, tc_peak):
+    """Named workloads of the other configurations. Each entry builds its inputs and
+    returns (call, report) where report(us) gives the line's figures."""
     import torch
-
-    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
-    out = {}
 
     def bf16(bits):
         return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
 
-    # odd-width dequant check (4096, 4095) -> bf16
-    c = workloads.decode_case(*workloads.ODD_DEQUANT_SHAPE)
-    codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
-    N, K = workloads.ODD_DEQUANT_SHAPE
-    o = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
-    t = time_calls(lambda: w4.dequantize(codes, scales, K, torch.bfloat16, out=o), 20, flush)
-    nb = payload(N, K) + 2 * N * K
-    out["dequant_4096x4095_bf16"] = {"us": 1e3 * t, "gbs": nb / t / 1e6, "frac_hbm": nb / t / 1e6 / hbm_peak}
-
-    # quantize (14336, 4096)
-    N, K = workloads.BATCHED_SHAPE
-    c = workloads.decode_case(N, K, M=64, config=3, bias=True)
-    W = torch.from_numpy(c["W"]).to(dev)
-    t = time_calls(lambda: w4.quantize_rtn(W, status=torch.zeros(1, dtype=torch.int32, device=dev)), 10, flush)
-    nb = 4 * N * K + payload(N, K)
-    out["quantize_14336x4096"] = {"us": 1e3 * t, "gbs": nb / t / 1e6, "frac_hbm": nb / t / 1e6 / hbm_peak}
-
-    # batched decode M in {8, 16, 32, 64}
-    codes, scales = w4.quantize_rtn(W)
-    del W
-    bias = torch.from_numpy(c["bias"]).to(dev)
-    xall = bf16(c["x_bits"])
-    for M in workloads.BATCHED_M:
-        x = xall[:M].contiguous()
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        t = time_calls(lambda: w4.linear(x, codes, scales, K, bias=bias, out=y), 30, flush)
-        fl = 2.0 * M * N * K
-        out[f"batched_M{M}_14336x4096"] = {"us": 1e3 * t, "weight_gbs": payload(N, K) / t / 1e6,
-                                           "frac_hbm": payload(N, K) / t / 1e6 / hbm_peak,
-                                           "tflops": fl / t / 1e9}
-
-    # prefill GEMMs
-    for M, N, K in workloads.PREFILL_SHAPES:
-        c = workloads.decode_case(N, K, M=M, config=4)
+    def dequant_odd():
+        N, K = workloads.ODD_DEQUANT_SHAPE
+        c = workloads.decode_case(N, K)
         codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
-        x = bf16(c["x_bits"])
-        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        t = time_calls(lambda: w4.linear(x, codes, scales, K, out=y), 5, flush)
-        fl = 2.0 * M * N * K
-        out[f"prefill_{M}x{N}x{K}"] = {"us": 1e3 * t, "tflops": fl / t / 1e9, "frac_tensor": fl / t / 1e9 / tc_peak}
-        del x, y, codes, scales
+        o = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        nb = payload(N, K) + 2 * N * K
+        return (lambda: w4.dequantize(codes, scales, K, torch.bfloat16, out=o),
+                lambda us: {"us": us, "gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
 
-    # asymmetric act-order, N=11008 K=4096 group 128
+    def quantize():
+        N, K = workloads.BATCHED_SHAPE
+        c = workloads.decode_case(N, K, M=1, config=3, bias=True)
+        W = torch.from_numpy(c["W"]).to(dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        nb = 4 * N * K + payload(N, K)
+        return (lambda: w4.quantize_rtn(W, status=st),
+                lambda us: {"us": us, "gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
+
+    def batched(M):
+        def make():
+            N, K = workloads.BATCHED_SHAPE
+            c = workloads.decode_case(N, K, M=M, config=3, bias=True)
+            codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
+            bias = torch.from_numpy(c["bias"]).to(dev)
+            x = bf16(c["x_bits"])
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            fl = 2.0 * M * N * K
+            return (lambda: w4.linear(x, codes, scales, K, bias=bias, out=y),
+                    lambda us: {"us": us, "weight_gbs": payload(N, K) / us / 1e3,
+                                "frac_hbm": payload(N, K) / us / 1e3 / hbm_peak, "tflops": fl / us / 1e6})
+        return make
+
+    def prefill(M, N, K):
+        def make():
+            c = workloads.decode_case(N, K, M=M, config=4)
+            codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
+            x = bf16(c["x_bits"])
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            fl = 2.0 * M * N * K
+            return (lambda: w4.linear(x, codes, scales, K, out=y),
+                    lambda us: {"us": us, "tflops": fl / us / 1e6, "frac_tensor": fl / us / 1e6 / tc_peak})
+        return make
+
+    def asym(M):
+        def make():
+            a = workloads.asym_random_codes(M)
+            gi = torch.from_numpy(a["g_idx"]).to(dev)
+            sc, perm = w4.asym_prepare(torch.from_numpy(a["codes"]).to(dev), gi, a["K"], a["n_groups"])
+            s = torch.from_numpy(a["scales"]).to(dev)
+            z = torch.from_numpy(a["zeros"]).to(dev)
+            x = bf16(a["x_bits"])
+            b = torch.from_numpy(a["bias"]).to(dev)
+            y = torch.empty((M, a["N"]), dtype=torch.bfloat16, device=dev)
+            nb = a["codes"].size + 4 * a["scales"].size + a["zeros"].size + 4 * a["K"]
+            fl = 2.0 * M * a["N"] * a["K"]
+            return (lambda: w4.linear_asym_gidx(x, sc, s, z, gi, perm=perm, bias=b, out=y),
+                    lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak,
+                                "tflops": fl / us / 1e6})
+        return make
+
+    w = {"dequant_4096x4095_bf16": dequant_odd, "quantize_14336x4096": quantize}
+    for M in workloads.BATCHED_M:
+        w[f"batched_M{M}_14336x4096"] = batched(M)
+    for M, N, K in workloads.PREFILL_SHAPES:
+        w[f"prefill_{M}x{N}x{K}"] = prefill(M, N, K)
     for M in workloads.ASYM_M:
-        a = workloads.asym_random_codes(M)
-        gi = torch.from_numpy(a["g_idx"]).to(dev)
-        sc, perm = w4.asym_prepare(torch.from_numpy(a["codes"]).to(dev), gi, a["K"], a["n_groups"])
-        s = torch.from_numpy(a["scales"]).to(dev)
-        z = torch.from_numpy(a["zeros"]).to(dev)
-        x = bf16(a["x_bits"])
-        b = torch.from_numpy(a["bias"]).to(dev)
-        y = torch.empty((M, a["N"]), dtype=torch.bfloat16, device=dev)
-        t = time_calls(lambda: w4.linear_asym_gidx(x, sc, s, z, gi, perm=perm, bias=b, out=y), 20, flush)
-        nb = a["codes"].size + 4 * a["scales"].size + a["zeros"].size + 4 * a["K"]
-        fl = 2.0 * M * a["N"] * a["K"]
-        out[f"asym_M{M}_11008x4096_g128"] = {"us": 1e3 * t, "weight_gbs": nb / t / 1e6,
-                                             "frac_hbm": nb / t / 1e6 / hbm_peak, "tflops": fl / t / 1e9}
+        w[f"asym_M{M}_11008x4096_g128"] = asym(M)
+    return w
+
+
+def run_detail(w4, dev, hbm_peak, tc_peak, only=None, iters=None, warmup=2):
+    """Time each named workload with CUDA events per call and a 256 MiB L2 flush between
+    calls (outside the timed events); report the median call."""
+    import torch
+
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    out = {}
+    for name, make in detail_workloads(w4, dev, hbm_peak, tc_peak).items():
+        if only is not None and name != only:
+            continue
+        call, report = make()
+        n = iters if iters is not None else (5 if name.startswith("prefill") else 20)
+        for _ in range(warmup):
+            call()
+        out[name] = report(1e3 * time_calls(call, n, flush))
+        del call
+        torch.cuda.empty_cache()
     return out
 
 

@@ -11,9 +11,11 @@
 //   * consumer warps own 32-column chunks (lane = chunk = one scale group = 16 code bytes),
 //     hold their activation chunk in registers for the whole kernel, and read the codes of
 //     each row from shared memory (512 contiguous bytes per warp instruction, conflict
-//     free). Each nibble becomes an exact fp32 integer (LOP3 + PRMT into the low byte of
-//     2^23, one exact fp32x2 subtract per pair) and meets the fp32 activations in fp32x2
-//     FMAs; the group scale multiplies the fp32 partial. The warps that together cover all chunks of a row form a group; with
+//     free). Nibble pairs become exact bf16x2 integers (one LOP3 each: the nibble drops into
+//     the mantissa of 128.0, whose ulp is 1; one exact bf16x2 FMA removes the offset) and
+//     meet the activations in sm_100 mixed-precision FMAs (bf16 x bf16 + fp32, full rate,
+//     the product is exact) in four independent chains; the group scale multiplies the fp32
+//     partial. The warps that together cover all chunks of a row form a group; with
 //     short rows several groups split the slots round-robin;
 //   * per slot, the group reduces 8 rows across lanes (transposing butterfly) and across
 //     its warps (shared memory, fixed order: deterministic), writes y and frees the slot.
@@ -26,13 +28,13 @@ namespace w4i {
 
 namespace {
 
-constexpr int kConsumerWarps = 16;
-constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kMaxConsumerWarps = 28;
 constexpr int kMaxSlots = 16;
 constexpr int kMaxCpl = 1;  // chunks per lane (K <= 16384)
 constexpr int kSmemBudget = 216 * 1024;
 
 struct StreamGeom {
+  int nw;           // consumer warps of the launch (24 or 28)
   int64_t P;        // code bytes per row
   int64_t SG;       // scale (and zero) columns per row
   int slot_bytes;   // 8 rows of codes + scales (+ zeros)
@@ -42,15 +44,16 @@ struct StreamGeom {
   int wg;           // warps per group: ceil(C / 32), at most 16
   int ngroups;      // 16 / wg
   int cpl;          // chunks per lane
+  int spg;          // slots per group (each group walks its own ring)
   int x_vec;        // 16-byte activation loads allowed
 };
 
 // Shared-memory tail after the slots: reduction buffers, barriers and the abort flag.
-constexpr int kRedBytes = 2 * kConsumerWarps * kGemvRows * 2 * 4;
+constexpr int kRedBytes = 2 * kMaxConsumerWarps * kGemvRows * 2 * 4;
 constexpr int kTailBytes = kRedBytes + 2 * kMaxSlots * 8 + 16;
 
-template <int MT, bool ASYM, int CPL>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int MT, bool ASYM, int CPL, int NW>
+__global__ void __launch_bounds__(32 * (NW + 1), 1)
     gemv_stream_kernel(const LinearParams p, const StreamGeom g, int32_t *err) {
   extern __shared__ __align__(128) uint8_t smem[];
   float *red = reinterpret_cast<float *>(smem + static_cast<size_t>(g.nslots) * g.slot_bytes);
@@ -79,8 +82,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- producer: one thread streams the CTA's rows through the slot ring ----
     if (lane == 0) {
       for (int s = 0; s < nstages; ++s) {
-        const int slot = s % g.nslots;
-        const uint32_t ph = static_cast<uint32_t>(s / g.nslots) & 1u;
+        // stage s belongs to group s % ngroups, which walks its own ring of spg slots
+        const int kq = s / g.ngroups;
+        const int slot = (s % g.ngroups) * g.spg + kq % g.spg;
+        const uint32_t ph = static_cast<uint32_t>(kq / g.spg) & 1u;
         if (!mbar_wait(&empty[slot], ph ^ 1u, abort_flag, err)) break;
         const int64_t r0 = row_begin + static_cast<int64_t>(s) * kGemvRows;
         const int64_t nr = (row_end - r0) < kGemvRows ? (row_end - r0) : kGemvRows;
@@ -102,16 +107,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int grp = cw / g.wg, wig = cw % g.wg;
   if (grp >= g.ngroups) return;
 
-  uint64_t xf[CPL][MT][16];
+  uint32_t xp[CPL][MT][16];
   int64_t chunk[CPL];
   int64_t cgroup[CPL];  // asym: scale column of the chunk
   bool mixed[CPL];
 #pragma unroll
   for (int j = 0; j < CPL; ++j) {
     chunk[j] = static_cast<int64_t>(wig) * 32 + lane + static_cast<int64_t>(j) * g.wg * 32;
-#pragma unroll
-    for (int m = 0; m < MT; ++m)
-      load_x_chunk_f32(p.x, m, M, K, 32 * chunk[j], g.x_vec != 0, ASYM ? p.perm : nullptr, xf[j][m]);
+    load_x_chunk<MT>(p.x, M, K, 32 * chunk[j], g.x_vec != 0, ASYM ? p.perm : nullptr, xp[j]);
     cgroup[j] = 0;
     mixed[j] = false;
     if (ASYM && chunk[j] < C) {
@@ -126,8 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bar_threads = 32 * g.wg;
   int buf = 0;
   for (int s = grp; s < nstages; s += g.ngroups) {
-    const int slot = s % g.nslots;
-    const uint32_t ph = static_cast<uint32_t>(s / g.nslots) & 1u;
+    const int kq = s / g.ngroups;
+    const int slot = grp * g.spg + kq % g.spg;
+    const uint32_t ph = static_cast<uint32_t>(kq / g.spg) & 1u;
     mbar_wait(&full[slot], ph, abort_flag, err);  // on failure: finish the pass on stale data
     const int64_t r0 = row_begin + static_cast<int64_t>(s) * kGemvRows;
     const int nr = static_cast<int>((row_end - r0) < kGemvRows ? (row_end - r0) : kGemvRows);
@@ -152,14 +156,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float scale = ss[r * g.SG + chunk[j]];
 #pragma unroll
               for (int m = 0; m < MT; ++m)
-                acc[r][m] = fmaf(f32x2_sum(dot_chunk_f32(cw4, xf[j][m], 0x08080808u, neg_magic2(8u), 0ull)),
-                                 scale, acc[r][m]);
+                acc[r][m] = fmaf(dot_chunk_ilp(cw4, xp[j][m], 0x43084308u, 0x43084308u), scale, acc[r][m]);
             } else if (!mixed[j]) {
               const float scale = ss[r * g.SG + cgroup[j]];
               const uint32_t z = static_cast<uint32_t>(static_cast<uint8_t>(sz[r * g.SG + cgroup[j]])) & 15u;
 #pragma unroll
               for (int m = 0; m < MT; ++m)
-                acc[r][m] = fmaf(f32x2_sum(dot_chunk_f32(cw4, xf[j][m], 0u, neg_magic2(z), 0ull)), scale,
+                acc[r][m] = fmaf(dot_chunk_ilp(cw4, xp[j][m], 0x43004300u, (0x4300u | z) * 0x00010001u), scale,
                                  acc[r][m]);
             } else {
               // sorted columns of two groups share this chunk: per-column scale and zero
@@ -175,8 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const float w = __fmul_rn(static_cast<float>(u - sz[r * g.SG + gg]), ss[r * g.SG + gg]);
 #pragma unroll
                   for (int m = 0; m < MT; ++m) {
-                    const uint64_t pair = xf[j][m][4 * t + (e >> 1)];
-                    acc[r][m] = fmaf(__uint_as_float(static_cast<uint32_t>((e & 1) ? (pair >> 32) : pair)), w,
+                    const uint32_t pair = xp[j][m][4 * t + (e & 3)];
+                    acc[r][m] = fmaf(__uint_as_float((e < 4 ? (pair & 0xFFFFu) : (pair >> 16)) << 16), w,
                                      acc[r][m]);
                   }
                 }
@@ -187,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
-    float *rb = red + buf * (kConsumerWarps * kGemvRows * 2);
+    float *rb = red + buf * (kMaxConsumerWarps * kGemvRows * 2);
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       float v[kGemvRows];
@@ -243,7 +246,11 @@ bool make_geom(const LinearParams &p, StreamGeom *g) {
   const uintptr_t align = reinterpret_cast<uintptr_t>(p.codes) | reinterpret_cast<uintptr_t>(p.scales) |
                           (p.asym ? reinterpret_cast<uintptr_t>(p.zeros) : 0);
   if (align % 16 != 0) return false;
-  const int64_t wg = (C + 31) / 32 < kConsumerWarps ? (C + 31) / 32 : kConsumerWarps;
+  const int64_t wg0 = (C + 31) / 32;
+  if (wg0 > kMaxConsumerWarps) return false;
+  // 24 consumer warps when rows need at most 4 warps, else 28 (two groups of up to 14)
+  const int nw = wg0 <= 4 ? 24 : 28;
+  const int64_t wg = wg0;
   const int64_t cpl = (C + wg * 32 - 1) / (wg * 32);
   if (cpl > kMaxCpl) return false;
   const int64_t codes_b = kGemvRows * g->P;
@@ -255,18 +262,23 @@ bool make_geom(const LinearParams &p, StreamGeom *g) {
   g->slot_bytes = static_cast<int>(slot);
   g->scales_off = static_cast<int>(codes_b);
   g->zeros_off = static_cast<int>(codes_b + scales_b);
-  g->nslots = static_cast<int>(nslots < kMaxSlots ? nslots : kMaxSlots);
+  const int64_t ns = nslots < kMaxSlots ? nslots : kMaxSlots;
+  int64_t ngroups = nw / wg < 8 ? nw / wg : 8;  // named barriers 1..8
+  if (ngroups > ns / 2) ngroups = ns / 2;
   g->wg = static_cast<int>(wg);
-  g->ngroups = static_cast<int>(kConsumerWarps / wg < 8 ? kConsumerWarps / wg : 8);  // named barriers 1..8
+  g->ngroups = static_cast<int>(ngroups);
+  g->spg = static_cast<int>(ns / ngroups);
+  g->nslots = static_cast<int>(ngroups * g->spg);
   g->cpl = static_cast<int>(cpl);
   g->x_vec = (K % 8 == 0) && (reinterpret_cast<uintptr_t>(p.x) % 16 == 0);
+  g->nw = nw;
   return true;
 }
 
-template <int MT, bool ASYM, int CPL>
+template <int MT, bool ASYM, int CPL, int NW>
 cudaError_t launch_typed(const LinearParams &p, const StreamGeom &g, int32_t *err, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(g.nslots) * g.slot_bytes + kTailBytes;
-  auto kern = gemv_stream_kernel<MT, ASYM, CPL>;
+  auto kern = gemv_stream_kernel<MT, ASYM, CPL, NW>;
   static bool attr_set = false;
   if (!attr_set) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBudget);
@@ -275,7 +287,7 @@ cudaError_t launch_typed(const LinearParams &p, const StreamGeom &g, int32_t *er
   }
   int64_t grid = (p.N + kGemvRows - 1) / kGemvRows;
   if (grid > sm_count()) grid = sm_count();
-  kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(p, g, err);
+  kern<<<static_cast<unsigned>(grid), 32 * (NW + 1), smem, stream>>>(p, g, err);
   return cudaGetLastError();
 }
 
@@ -289,7 +301,9 @@ bool gemv_stream_supports(const LinearParams &p) {
 cudaError_t launch_gemv_stream(const LinearParams &p, int32_t *err, cudaStream_t stream) {
   StreamGeom g;
   if (!make_geom(p, &g)) return cudaErrorNotSupported;
-  return p.asym ? launch_typed<1, true, 1>(p, g, err, stream) : launch_typed<1, false, 1>(p, g, err, stream);
+  if (g.nw == 24)
+    return p.asym ? launch_typed<1, true, 1, 24>(p, g, err, stream) : launch_typed<1, false, 1, 24>(p, g, err, stream);
+  return p.asym ? launch_typed<1, true, 1, 28>(p, g, err, stream) : launch_typed<1, false, 1, 28>(p, g, err, stream);
 }
 
 }  // namespace w4i

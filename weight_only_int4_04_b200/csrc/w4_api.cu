@@ -2,6 +2,7 @@
 // selection and error reporting. No device memory is allocated here; the only device state
 // is the static status words below (one per loaded library, shared by every call).
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <vector>
 
@@ -44,12 +45,24 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
   int32_t *err = nullptr;
   const w4_status st = symbol_ptr(&err, g_device_error);
   if (st != W4_OK) return st;
-  // M dispatch: streaming GEMV for M = 1, the register GEMV for M <= 4, the tcgen05 GEMM
-  // above that; the generic kernel takes whatever the fast paths cannot (odd widths,
-  // unaligned rows, unsorted act-order maps).
+  // M dispatch: M = 1 -> the register-streaming GEMV; M <= 16 -> the tensor-core decode
+  // kernel (bulk-copy slot ring, mma.sync); larger M -> the tcgen05 GEMM; the other GEMV
+  // kernels and the generic kernel take the shapes the fast paths cannot (unaligned rows,
+  // odd widths, unsorted act-order maps). W4_GEMV=stream|mma picks the alternative M = 1
+  // kernels (for comparisons only).
+  static const int m1_kernel = [] {
+    const char *v = getenv("W4_GEMV");
+    if (v != nullptr && strcmp(v, "stream") == 0) return 1;
+    if (v != nullptr && strcmp(v, "mma") == 0) return 2;
+    return 0;
+  }();
   cudaError_t e;
-  if (w4i::gemv_stream_supports(p)) {
+  if (m1_kernel == 0 && w4i::gemv_rows_supports(p)) {
+    e = w4i::launch_gemv_rows(p, stream);
+  } else if (m1_kernel != 2 && w4i::gemv_stream_supports(p)) {
     e = w4i::launch_gemv_stream(p, err, stream);
+  } else if (w4i::gemv_mma_supports(p)) {
+    e = w4i::launch_gemv_mma(p, err, stream);
   } else if (w4i::gemv_supports(p)) {
     e = w4i::launch_gemv(p, stream);
   } else if (p.M > 4 && w4i::gemm_tc_supports(p)) {

@@ -73,6 +73,23 @@ __device__ __forceinline__ float dot_chunk(const uint4 cw, const uint32_t *xp, u
   return acc;
 }
 
+// Same sum with four independent accumulators (one per code word) so that consecutive FMAs
+// do not wait on each other; the partial sums are added at the end.
+__device__ __forceinline__ float dot_chunk_ilp(const uint4 cw, const uint32_t *xp, uint32_t magic,
+                                               uint32_t offset) {
+  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t w = words[t];
+    acc[t] = fma2_bf16_f32(xp[4 * t + 0], bf16x2_sub(nib_pair_bf16(w, magic), offset), acc[t]);
+    acc[t] = fma2_bf16_f32(xp[4 * t + 1], bf16x2_sub(nib_pair_bf16(w >> 4, magic), offset), acc[t]);
+    acc[t] = fma2_bf16_f32(xp[4 * t + 2], bf16x2_sub(nib_pair_bf16(w >> 8, magic), offset), acc[t]);
+    acc[t] = fma2_bf16_f32(xp[4 * t + 3], bf16x2_sub(nib_pair_bf16(w >> 12, magic), offset), acc[t]);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 // Transposing butterfly: lane l ends with the warp-wide sum of row (l >> 2) & 7.
 __device__ __forceinline__ float reduce_rows8(float v[kGemvRows], int lane) {
 #pragma unroll

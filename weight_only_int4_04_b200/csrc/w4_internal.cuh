@@ -49,6 +49,13 @@ bool gemv_supports(const LinearParams &p);
 // `err` is the library's device error word (bounded waits report W4_ERR_TIMEOUT there).
 cudaError_t launch_gemv_stream(const LinearParams &p, int32_t *err, cudaStream_t stream);
 bool gemv_stream_supports(const LinearParams &p);
+// Register-streaming decode GEMV (M = 1): every lane prefetches its own code rows.
+cudaError_t launch_gemv_rows(const LinearParams &p, cudaStream_t stream);
+bool gemv_rows_supports(const LinearParams &p);
+// Small-M linear (M <= 16) on register-fed tensor cores (mma.sync), streaming rows through a
+// bulk-copy slot ring; the main decode path.
+cudaError_t launch_gemv_mma(const LinearParams &p, int32_t *err, cudaStream_t stream);
+bool gemv_mma_supports(const LinearParams &p);
 // Tensor-core GEMM (tcgen05, TMA, TMEM) for larger M; symmetric codes, aligned rows.
 cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t stream);
 bool gemm_tc_supports(const LinearParams &p);
@@ -79,10 +86,11 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// bf16x2 subtraction (exact for the small integers it is used on).
+// bf16x2 a - b computed as fma(a, 1, -b) (fma.rn.bf16x2, a native sm_80+ instruction;
+// exact for the small integers it is used on).
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(0x3F803F80u), "r"(b ^ 0x80008000u));
   return d;
 }
 
