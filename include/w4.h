@@ -122,6 +122,12 @@ w4_status w4_linear(const void *x, int64_t M, const uint8_t *codes, const float 
 /* Workspace bytes w4_linear needs for this shape (0 = none). */
 size_t w4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
+/* Workspace bytes w4_linear_asym_gidx uses for this shape when its codes are prepared
+ * (perm given): for M above the decode sizes the activations are gathered through perm into
+ * the workspace (M * K bf16, rounded up to 256 bytes) and a tensor-core GEMM runs. A call
+ * given less (or no) workspace still succeeds on a slower kernel. */
+size_t w4_linear_asym_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t n_groups);
+
 /*
  * w4_asym_prepare -- one-time act-order preparation of an asymmetric weight.
  * Sorts the columns by group (stable: columns of one group keep their order) and writes
@@ -145,7 +151,9 @@ w4_status w4_asym_prepare(const uint8_t *codes_in, const int32_t *g_idx, int64_t
  *            column order; if perm != NULL they are the codes_out of w4_asym_prepare.
  *   scales   float32 [N, n_groups]; zeros int8 [N, n_groups] in [0, 15];
  *   g_idx    int32 [K]: group of ORIGINAL column k;  perm  int32 [K] or NULL.
- *   x, bias, y, y_dtype, workspace: as w4_linear; the same tolerance holds.
+ *   x, bias, y, y_dtype: as w4_linear; the same tolerance holds.
+ *   workspace  NULL or 256-byte aligned device memory of w4_linear_asym_workspace_bytes(...)
+ *              bytes (W4_ERR_WORKSPACE if misaligned); calls sharing it must not overlap.
  */
 w4_status w4_linear_asym_gidx(const void *x, int64_t M, const uint8_t *codes,
                               const float *scales, const int8_t *zeros, const int32_t *g_idx,

@@ -29,23 +29,18 @@ STATUS = {
 DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2, torch.float64: 3}
 
 EXPORTS = (
-    "w4_quantize_rtn", "w4_dequantize", "w4_linear", "w4_linear_workspace_bytes",
+    "w4_quantize_rtn", "w4_dequantize", "w4_linear", "w4_linear_workspace_bytes", "w4_linear_asym_workspace_bytes",
     "w4_asym_prepare", "w4_linear_asym_gidx", "w4_validate", "w4_validate_asym",
     "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
 )
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m weight_only_int4_04_b200.build` "
-        "(there is no CPU fallback)")
-
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
-lib = ctypes.CDLL(LIB_PATH)
 _SIGS = {
     "w4_quantize_rtn": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
     "w4_dequantize": [_vp, _vp, _i64, _i64, _i32, _i32, _vp, _vp],
     "w4_linear": [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _vp, _sz, _vp],
     "w4_linear_workspace_bytes": [_i64, _i64, _i64],
+    "w4_linear_asym_workspace_bytes": [_i64, _i64, _i64, _i64],
     "w4_asym_prepare": [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
     "w4_linear_asym_gidx": [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp, _sz,
                             _vp],
@@ -56,21 +51,44 @@ _SIGS = {
     "w4_status_string": [_i32],
     "w4_version": [],
 }
-for _name, _args in _SIGS.items():
-    _f = getattr(lib, _name)
-    _f.argtypes = _args
-    _f.restype = ctypes.c_int
-lib.w4_linear_workspace_bytes.restype = ctypes.c_size_t
-lib.w4_status_string.restype = ctypes.c_char_p
+_lib = None
+
+
+def _load():
+    """Load libw4.so on first use; raise loudly if it was never built (no CPU fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m weight_only_int4_04_b200.build` "
+                "(there is no CPU fallback)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, args in _SIGS.items():
+            f = getattr(handle, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        handle.w4_linear_workspace_bytes.restype = ctypes.c_size_t
+        handle.w4_linear_asym_workspace_bytes.restype = ctypes.c_size_t
+        handle.w4_status_string.restype = ctypes.c_char_p
+        _lib = handle
+    return _lib
+
+
+def __getattr__(name):
+    # `lib` is the loaded library; resolved lazily so that the build module can be imported
+    # (and run) before the library exists.
+    if name == "lib":
+        return _load()
+    raise AttributeError(name)
 
 
 class W4Error(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         self.name = STATUS.get(status, str(status))
-        msg = lib.w4_status_string(status).decode()
+        msg = _load().w4_status_string(status).decode()
         if self.name == "CUDA":
-            msg += f" (cudaError {lib.w4_last_cuda_error()})"
+            msg += f" (cudaError {_load().w4_last_cuda_error()})"
         super().__init__(f"{where}: {self.name}: {msg}")
 
 
@@ -105,7 +123,7 @@ def quantize_rtn(W: torch.Tensor, status: torch.Tensor | None = None):
     N, K = W.shape
     codes = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=W.device)
     scales = torch.empty((N, (K + 31) // 32), dtype=torch.float32, device=W.device)
-    _check(lib.w4_quantize_rtn(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(status), _stream()),
+    _check(_load().w4_quantize_rtn(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(status), _stream()),
            "w4_quantize_rtn")
     return codes, scales
 
@@ -119,17 +137,22 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, K: int, out_dtype=torc
         raise ValueError("unsupported output dtype")
     if out is None:
         out = torch.empty((N, K), dtype=out_dtype, device=codes.device)
-    _check(lib.w4_dequantize(_ptr(codes), _ptr(scales), N, K, format_version, DTYPES[out_dtype], _ptr(out),
+    _check(_load().w4_dequantize(_ptr(codes), _ptr(scales), N, K, format_version, DTYPES[out_dtype], _ptr(out),
                              _stream()), "w4_dequantize")
     return out
 
 
 def workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(lib.w4_linear_workspace_bytes(M, N, K))
+    return int(_load().w4_linear_workspace_bytes(M, N, K))
 
 
-def _workspace(M, N, K, device, workspace):
-    need = workspace_bytes(M, N, K)
+def asym_workspace_bytes(M: int, N: int, K: int, n_groups: int) -> int:
+    return int(_load().w4_linear_asym_workspace_bytes(M, N, K, n_groups))
+
+
+def _workspace(M, N, K, device, workspace, need=None):
+    if need is None:
+        need = workspace_bytes(M, N, K)
     if need == 0:
         return None, 0
     if workspace is None or workspace.numel() * workspace.element_size() < need:
@@ -152,7 +175,7 @@ def linear(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, K: int | 
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
     ws, wsb = _workspace(M, N, K, x.device, workspace)
-    _check(lib.w4_linear(_ptr(x), M, _ptr(codes), _ptr(scales), N, K, _ptr(bias), _ptr(out),
+    _check(_load().w4_linear(_ptr(x), M, _ptr(codes), _ptr(scales), N, K, _ptr(bias), _ptr(out),
                          DTYPES[out.dtype], _ptr(ws), wsb, _stream()), "w4_linear")
     return out
 
@@ -163,7 +186,7 @@ def asym_prepare(codes: torch.Tensor, g_idx: torch.Tensor, K: int, n_groups: int
     N = codes.shape[0]
     out = torch.empty_like(codes)
     perm = torch.empty(K, dtype=torch.int32, device=codes.device)
-    _check(lib.w4_asym_prepare(_ptr(codes), _ptr(g_idx), N, K, n_groups, _ptr(out), _ptr(perm), _stream()),
+    _check(_load().w4_asym_prepare(_ptr(codes), _ptr(g_idx), N, K, n_groups, _ptr(out), _ptr(perm), _stream()),
            "w4_asym_prepare")
     return out, perm
 
@@ -181,8 +204,9 @@ def linear_asym_gidx(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
     N, G = scales.shape
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=x.device)
-    ws, wsb = _workspace(M, N, K, x.device, workspace)
-    _check(lib.w4_linear_asym_gidx(_ptr(x), M, _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), _ptr(perm),
+    need = asym_workspace_bytes(M, N, K, G) if perm is not None else 0
+    ws, wsb = _workspace(M, N, K, x.device, workspace, need)
+    _check(_load().w4_linear_asym_gidx(_ptr(x), M, _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), _ptr(perm),
                                    N, K, G, _ptr(bias), _ptr(out), DTYPES[out.dtype], _ptr(ws), wsb,
                                    _stream()), "w4_linear_asym_gidx")
     return out
@@ -191,14 +215,14 @@ def linear_asym_gidx(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
 def validate(codes: torch.Tensor, scales: torch.Tensor, K: int, format_version: int = 2) -> str:
     """LoopQ content checks on the device; returns the status name ("OK" if valid)."""
     _need_cuda(codes, scales)
-    return STATUS[lib.w4_validate(_ptr(codes), _ptr(scales), codes.shape[0], K, format_version, _stream())]
+    return STATUS[_load().w4_validate(_ptr(codes), _ptr(scales), codes.shape[0], K, format_version, _stream())]
 
 
 def validate_asym(codes, scales, zeros, g_idx, K: int) -> str:
     _need_cuda(codes, scales, zeros, g_idx)
-    return STATUS[lib.w4_validate_asym(_ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), codes.shape[0], K,
+    return STATUS[_load().w4_validate_asym(_ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), codes.shape[0], K,
                                        scales.shape[1], _stream())]
 
 
 def device_error() -> str:
-    return STATUS[lib.w4_device_error()]
+    return STATUS[_load().w4_device_error()]

@@ -37,14 +37,24 @@ constexpr int kDequantWarp0 = 2;
 constexpr int A_BYTES = BM_W * BK * 2;    // 16 KB
 constexpr int B_BYTES = BN_X * BK * 2;    // 32 KB
 constexpr int C_BYTES = BM_W * (BK / 2);  // 4 KB of codes
-constexpr int S_BYTES = BM_W * 4 * 4;     // 2 KB: 4 scale groups per row (two stages' worth)
+constexpr int S_BYTES = BM_W * 4 * 4;     // 2 KB: 4 scale columns per row
+constexpr int Z_BYTES = BM_W * 16;        // 2 KB: 16 zero-point columns per row (asymmetric)
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
 constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
 constexpr int OFF_S = OFF_C + STAGES * C_BYTES;
-constexpr int OFF_BAR = OFF_S + STAGES * S_BYTES;
-constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + 1 KB alignment slack
-constexpr uint32_t TX_BYTES = B_BYTES + C_BYTES + S_BYTES;
+constexpr int OFF_Z = OFF_S + STAGES * S_BYTES;
+template <bool ASYM>
+__host__ __device__ constexpr int off_gstage() { return ASYM ? OFF_Z + STAGES * Z_BYTES : OFF_Z; }
+constexpr int kMaxStagesAsym = 512;        // K <= 32768 on the asymmetric path
+template <bool ASYM>
+__host__ __device__ constexpr int off_bar() { return off_gstage<ASYM>() + (ASYM ? 2 * kMaxStagesAsym : 0); }
+template <bool ASYM>
+__host__ __device__ constexpr int smem_bytes() { return off_bar<ASYM>() + 256 + 1024; }  // barriers + 1 KB alignment slack
+static_assert(smem_bytes<true>() <= 227 * 1024, "asymmetric GEMM exceeds the shared-memory budget");
+static_assert(smem_bytes<false>() <= 227 * 1024, "GEMM exceeds the shared-memory budget");
+template <bool ASYM>
+__host__ __device__ constexpr uint32_t tx_bytes() { return B_BYTES + C_BYTES + S_BYTES + (ASYM ? Z_BYTES : 0); }
 constexpr uint32_t TMEM_COLS = BN_X;
 
 struct TcParams {
@@ -52,16 +62,26 @@ struct TcParams {
   void *y;
   int64_t M, N, K;
   int y_dtype;
+  // asymmetric act-order only: columns are sorted; the stage table maps each 64-column K
+  // block to its scale column (or -1 when the block spans two groups)
+  const int32_t *g_idx;
+  const int32_t *perm;
+  const float *scales;
+  const int8_t *zeros;
+  int n_groups;
 };
 
+template <bool ASYM>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
-                   const __grid_constant__ CUtensorMap tmap_scales, const TcParams p, int32_t *err) {
+                   const __grid_constant__ CUtensorMap tmap_scales, const __grid_constant__ CUtensorMap tmap_zeros,
+                   const TcParams p, int32_t *err) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base (the 128-byte swizzle atoms must start on 1024-byte boundaries)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint64_t *full_load = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint64_t *full_load = reinterpret_cast<uint64_t *>(smem + off_bar<ASYM>());
+  int16_t *gstage = reinterpret_cast<int16_t *>(smem + off_gstage<ASYM>());
   uint64_t *full_a = full_load + STAGES;
   uint64_t *empty = full_a + STAGES;
   uint64_t *acc_full = empty + STAGES;
@@ -83,6 +103,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     mbar_fence_init();
   }
+  if (ASYM) {
+    // scale column of every 64-column K block of the sorted columns (-1: two groups)
+    for (int kb = threadIdx.x; kb < KB; kb += kThreads) {
+      const int64_t c0 = static_cast<int64_t>(kb) * BK;
+      const int64_t last = (c0 + BK - 1 < p.K) ? c0 + BK - 1 : p.K - 1;
+      const int32_t g0 = __ldg(p.g_idx + __ldg(p.perm + c0));
+      gstage[kb] = static_cast<int16_t>(g0 == __ldg(p.g_idx + __ldg(p.perm + last)) ? g0 : -1);
+    }
+  }
   if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -95,12 +124,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = kb % STAGES;
         const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err)) break;
-        mbar_arrive_expect_tx(&full_load[s], TX_BYTES);
+        mbar_arrive_expect_tx(&full_load[s], tx_bytes<ASYM>());
         tma_load_2d(smem + OFF_B + s * B_BYTES, &tmap_x, kb * BK, static_cast<int32_t>(m0), &full_load[s]);
         tma_load_2d(smem + OFF_C + s * C_BYTES, &tmap_codes, kb * (BK / 2), static_cast<int32_t>(n0),
                     &full_load[s]);
-        tma_load_2d(smem + OFF_S + s * S_BYTES, &tmap_scales, 4 * (kb / 2), static_cast<int32_t>(n0),
-                    &full_load[s]);
+        if (!ASYM) {
+          tma_load_2d(smem + OFF_S + s * S_BYTES, &tmap_scales, 4 * (kb / 2), static_cast<int32_t>(n0),
+                      &full_load[s]);
+        } else {
+          const int gs = gstage[kb] < 0 ? 0 : gstage[kb];
+          tma_load_2d(smem + OFF_S + s * S_BYTES, &tmap_scales, gs & ~3, static_cast<int32_t>(n0), &full_load[s]);
+          tma_load_2d(smem + OFF_Z + s * Z_BYTES, &tmap_zeros, gs & ~15, static_cast<int32_t>(n0), &full_load[s]);
+        }
       }
     }
   } else if (warp == 1) {
@@ -135,14 +170,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
       mbar_wait(&full_load[s], ph, abort_flag, err);
       const uint4 cw = *reinterpret_cast<const uint4 *>(smem + OFF_C + s * C_BYTES + r * 32 + 16 * half);
-      const float sc = reinterpret_cast<const float *>(smem + OFF_S + s * S_BYTES)[r * 4 + (kb & 1) * 2 + half];
-      const uint64_t scale2 = (static_cast<uint64_t>(__float_as_uint(sc)) << 32) | __float_as_uint(sc);
       const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+      float sc;
+      uint32_t xorc = 0x08080808u;
+      uint64_t nb2 = neg_bias_pair(8u);
+      int gs = 0;
+      if (!ASYM) {
+        sc = reinterpret_cast<const float *>(smem + OFF_S + s * S_BYTES)[r * 4 + (kb & 1) * 2 + half];
+      } else {
+        gs = gstage[kb];
+        const int gsc = gs < 0 ? 0 : gs;
+        sc = reinterpret_cast<const float *>(smem + OFF_S + s * S_BYTES)[r * 4 + (gsc & 3)];
+        const uint32_t z = static_cast<uint32_t>(
+            reinterpret_cast<const uint8_t *>(smem + OFF_Z + s * Z_BYTES)[r * 16 + (gsc & 15)]) & 15u;
+        xorc = 0u;
+        nb2 = neg_bias_pair(z);
+      }
+      const uint64_t scale2 = (static_cast<uint64_t>(__float_as_uint(sc)) << 32) | __float_as_uint(sc);
+      if (!ASYM || gs >= 0) {
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const uint4 v = dequant_word_bf16(words[t], scale2);
-        const uint32_t chunk = static_cast<uint32_t>(4 * half + t) ^ static_cast<uint32_t>(r & 7);
-        st_shared_v4(a_row + s * A_BYTES + chunk * 16, v);
+        for (int t = 0; t < 4; ++t) {
+          const uint4 v = dequant_word_bf16(words[t], scale2, xorc, nb2);
+          const uint32_t chunk = static_cast<uint32_t>(4 * half + t) ^ static_cast<uint32_t>(r & 7);
+          st_shared_v4(a_row + s * A_BYTES + chunk * 16, v);
+        }
+      } else {
+        // this K block spans two groups: per-column scale and zero from global memory
+        const int64_t n = n0 + r;
+#pragma unroll 1
+        for (int t = 0; t < 4; ++t) {
+          uint32_t packed[4];
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float wv[2];
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 2 * e2 + h2;
+              const int64_t col = static_cast<int64_t>(kb) * BK + 32 * half + 8 * t + e;
+              wv[h2] = 0.0f;
+              if (n < p.N && col < p.K) {
+                const int64_t gg = __ldg(p.g_idx + __ldg(p.perm + col));
+                const int u = static_cast<int>((words[t] >> (4 * e)) & 15u);
+                wv[h2] = __fmul_rn(static_cast<float>(u - p.zeros[n * p.n_groups + gg]),
+                                   p.scales[n * p.n_groups + gg]);
+              }
+            }
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(packed[e2]) : "f"(wv[1]), "f"(wv[0]));
+          }
+          const uint32_t chunk = static_cast<uint32_t>(4 * half + t) ^ static_cast<uint32_t>(r & 7);
+          st_shared_v4(a_row + s * A_BYTES + chunk * 16, make_uint4(packed[0], packed[1], packed[2], packed[3]));
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -216,35 +291,92 @@ bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uin
 }  // namespace
 
 bool gemm_tc_supports(const LinearParams &p) {
-  if (p.asym) return false;
   const int64_t P = (p.K + 1) / 2, G = (p.K + 31) / 32;
-  if (p.K % 8 != 0 || P % 16 != 0 || G % 4 != 0) return false;
-  const uintptr_t a = reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.codes) |
-                      reinterpret_cast<uintptr_t>(p.scales);
+  if (p.K % 8 != 0 || P % 16 != 0) return false;
+  if (!p.asym && G % 4 != 0) return false;
+  if (p.asym && (p.perm == nullptr || p.n_groups % 16 != 0 || (p.K + BK - 1) / BK > kMaxStagesAsym ||
+                 p.n_groups > 32767))
+    return false;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p.codes) | reinterpret_cast<uintptr_t>(p.scales) |
+                      (p.asym ? reinterpret_cast<uintptr_t>(p.zeros) : 0) |
+                      (p.asym ? 0 : reinterpret_cast<uintptr_t>(p.x));
   if (a % 16 != 0) return false;
   if ((p.M + BN_X - 1) / BN_X > 65535 || (p.N + BM_W - 1) / BM_W > 0x7fffffffLL) return false;
   return encode_fn() != nullptr;
 }
 
-cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t stream) {
+// x gathered through perm (act-order): xg[m][j] = x[m][perm[j]], eight columns per thread.
+__global__ void __launch_bounds__(256) gather_x_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                       const int32_t *__restrict__ perm, int64_t M, int64_t K,
+                                                       __nv_bfloat16 *__restrict__ xg) {
+  const int64_t units = M * (K / 8);
+  const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
+       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = u / (K / 8), j0 = (u % (K / 8)) * 8;
+    uint32_t v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = __ldg(xb + m * K + __ldg(perm + j0 + 2 * i));
+      const uint32_t hi = __ldg(xb + m * K + __ldg(perm + j0 + 2 * i + 1));
+      v[i] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4 *>(xg + m * K + j0) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+size_t gemm_tc_asym_workspace(int64_t M, int64_t K) {
+  return static_cast<size_t>(((M * K * 2 + 255) / 256) * 256);
+}
+
+cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t stream, void *workspace) {
   if (!gemm_tc_supports(p)) return cudaErrorNotSupported;
   const int64_t P = (p.K + 1) / 2, G = (p.K + 31) / 32;
-  CUtensorMap mx, mc, ms;
-  if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, BK, BN_X,
+  const __nv_bfloat16 *xsrc = p.x;
+  if (p.asym) {
+    // act-order: the activations are gathered once into the workspace in sorted column order
+    if (workspace == nullptr || reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return cudaErrorInvalidValue;
+    __nv_bfloat16 *xg = static_cast<__nv_bfloat16 *>(workspace);
+    int64_t blocks = (p.M * (p.K / 8) + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    gather_x_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.x, p.perm, p.M, p.K, xg);
+    xsrc = xg;
+  }
+  const int64_t SG = p.asym ? p.n_groups : G;
+  CUtensorMap mx, mc, ms, mz;
+  if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xsrc, p.K, p.M, p.K * 2, BK, BN_X,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.codes, P, p.N, P, BK / 2, BM_W, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.scales, G, p.N, G * 4, 4, BM_W,
+      !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.scales, SG, p.N, SG * 4, 4, BM_W,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr = true;
+  if (p.asym) {
+    if (!make_map_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.zeros, SG, p.N, SG, 16, BM_W, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  } else {
+    mz = ms;  // unused by the symmetric kernel
   }
-  TcParams tp{p.bias, p.y, p.M, p.N, p.K, p.y_dtype};
+  TcParams tp{p.bias, p.y, p.M, p.N, p.K, p.y_dtype, p.g_idx, p.perm, p.scales, p.zeros, p.n_groups};
   const dim3 grid(static_cast<unsigned>((p.N + BM_W - 1) / BM_W), static_cast<unsigned>((p.M + BN_X - 1) / BN_X));
-  gemm_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(mx, mc, ms, tp, err);
+  if (p.asym) {
+    static bool attr = false;
+    if (!attr) {
+      const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem_bytes<true>());
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    gemm_tc_kernel<true><<<grid, kThreads, smem_bytes<true>(), stream>>>(mx, mc, ms, mz, tp, err);
+  } else {
+    static bool attr = false;
+    if (!attr) {
+      const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem_bytes<false>());
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    gemm_tc_kernel<false><<<grid, kThreads, smem_bytes<false>(), stream>>>(mx, mc, ms, mz, tp, err);
+  }
   return cudaGetLastError();
 }
 

@@ -38,10 +38,16 @@ w4_status symbol_ptr(T **out, const T &sym) {
   return W4_OK;
 }
 
+// Tensor-core GEMM is used above this M (and whenever the decode kernels do not apply).
+constexpr int64_t kTcMinM = 17;
+
+// The asymmetric tensor-core path gathers x into the workspace; everything else needs none.
+bool asym_uses_tc(const w4i::LinearParams &p) {
+  return p.asym && p.M >= kTcMinM && w4i::gemm_tc_supports(p);
+}
+
 w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspace_bytes,
                      cudaStream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   int32_t *err = nullptr;
   const w4_status st = symbol_ptr(&err, g_device_error);
   if (st != W4_OK) return st;
@@ -65,8 +71,9 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
     e = w4i::launch_gemv_mma(p, err, stream);
   } else if (w4i::gemv_supports(p)) {
     e = w4i::launch_gemv(p, stream);
-  } else if (p.M > 4 && w4i::gemm_tc_supports(p)) {
-    e = w4i::launch_gemm_tc(p, err, stream);
+  } else if (p.M > 4 && w4i::gemm_tc_supports(p) &&
+             (!p.asym || (workspace != nullptr && workspace_bytes >= w4i::gemm_tc_asym_workspace(p.M, p.K)))) {
+    e = w4i::launch_gemm_tc(p, err, stream, workspace);
   } else {
     e = w4i::launch_linear_generic(p, stream);
   }
@@ -168,6 +175,12 @@ w4_status w4_linear(const void *x, int64_t M, const uint8_t *codes, const float 
   return run_linear(p, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t w4_linear_asym_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t n_groups) {
+  // act-order GEMMs above the decode sizes gather x through perm: M * K bf16
+  if (M < kTcMinM || K % 8 != 0 || n_groups % 16 != 0 || M < 1 || K < 1 || N < 1) return 0;
+  return w4i::gemm_tc_asym_workspace(M, K);
+}
+
 w4_status w4_asym_prepare(const uint8_t *codes_in, const int32_t *g_idx, int64_t N, int64_t K,
                           int64_t n_groups, uint8_t *codes_out, int32_t *perm, w4_stream_t stream) {
   if (!codes_in || !g_idx || !codes_out || !perm) return W4_ERR_NULL;
@@ -197,9 +210,9 @@ w4_status w4_linear_asym_gidx(const void *x, int64_t M, const uint8_t *codes, co
   if (!x || !codes || !scales || !zeros || !g_idx || !y) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || M < 1 || M > kMaxRows || n_groups < 1 || n_groups > K) return W4_ERR_SHAPE;
   if (y_dtype != W4_BF16 && y_dtype != W4_F32) return W4_ERR_DTYPE;
-  const size_t need = w4_linear_workspace_bytes(M, N, K);
-  if (need > 0 && (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256))
-    return W4_ERR_WORKSPACE;
+  // With codes sorted by w4_asym_prepare (perm given) the tensor-core path needs the
+  // workspace; without it a slower kernel serves the call (no error).
+  if (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % 256) return W4_ERR_WORKSPACE;
   w4i::LinearParams p{};
   p.x = static_cast<const __nv_bfloat16 *>(x);
   p.codes = codes;

@@ -56,9 +56,11 @@ bool gemv_rows_supports(const LinearParams &p);
 // bulk-copy slot ring; the main decode path.
 cudaError_t launch_gemv_mma(const LinearParams &p, int32_t *err, cudaStream_t stream);
 bool gemv_mma_supports(const LinearParams &p);
-// Tensor-core GEMM (tcgen05, TMA, TMEM) for larger M; symmetric codes, aligned rows.
-cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t stream);
+// Tensor-core GEMM (tcgen05, TMA, TMEM) for larger M, aligned rows. The asymmetric
+// act-order variant gathers x through perm into `workspace` (gemm_tc_asym_workspace bytes).
+cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t stream, void *workspace);
 bool gemm_tc_supports(const LinearParams &p);
+size_t gemm_tc_asym_workspace(int64_t M, int64_t K);
 
 // Validation flag bits (w4_validate reports them in the page's order).
 enum : uint32_t {

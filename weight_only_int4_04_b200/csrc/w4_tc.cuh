@@ -107,29 +107,36 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-// Eight signed nibbles of one code word (columns 8t .. 8t+7, even column low) -> eight
-// bf16 weights bf16(fp32(q * s)) in column order, packed as four bf16x2. Per column pair:
-// the nibble (xor 8) is placed in the low byte of the fp32 2^23 (PRMT), an exact fp32x2
-// subtract of 2^23 + 8 leaves q, one fp32x2 multiply by the scale rounds once, and the
-// pair is rounded to bf16 with round-to-nearest-even -- the same value w4_dequantize
-// produces for bf16 output.
-__device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, uint64_t scale2) {
-  const uint32_t lo = lop3_and_xor(w, 0x0F0F0F0Fu, 0x08080808u);       // even columns
-  const uint32_t hi = lop3_and_xor(w >> 4, 0x0F0F0F0Fu, 0x08080808u);  // odd columns
-  const uint64_t bias2 = 0xCB000008CB000008ull;                      // -(2^23 + 8), twice
+// Eight nibbles of one code word (columns 8t .. 8t+7, even column low) -> eight bf16
+// weights bf16(fp32(v * s)) in column order, packed as four bf16x2. Per column pair: the
+// nibble (xor 8 for signed codes) is placed in the low byte of the fp32 2^23 (PRMT), an
+// exact fp32x2 subtract of neg_bias2 = 2^23 + 8 (signed: leaves q) or 2^23 + z (unsigned:
+// leaves u - z) , one fp32x2 multiply by the scale rounds once, and the pair is rounded to
+// bf16 with round-to-nearest-even -- for signed codes the same value w4_dequantize produces
+// for bf16 output.
+__device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, uint64_t scale2, uint32_t xorc,
+                                                   uint64_t neg_bias2) {
+  const uint32_t lo = lop3_and_xor(w, 0x0F0F0F0Fu, xorc);       // even columns
+  const uint32_t hi = lop3_and_xor(w >> 4, 0x0F0F0F0Fu, xorc);  // odd columns
   uint32_t out[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t fe = prmt(lo, 0x00004B00u, 0x5440u | i);
     const uint32_t fo = prmt(hi, 0x00004B00u, 0x5440u | i);
     uint64_t v = (static_cast<uint64_t>(fo) << 32) | fe;
-    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(bias2));
+    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(neg_bias2));
     asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(scale2));
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
         : "=r"(out[i])
         : "f"(__uint_as_float(static_cast<uint32_t>(v >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(v))));
   }
   return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// -(2^23 + v) as a pair of fp32 bit patterns (v in [0, 15]).
+__device__ __forceinline__ uint64_t neg_bias_pair(uint32_t v) {
+  const uint64_t f = 0xCB000000u | v;
+  return (f << 32) | f;
 }
 
 }  // namespace w4i
