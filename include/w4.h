@@ -162,6 +162,30 @@ w4_status w4_linear_asym_gidx(const void *x, int64_t M, const uint8_t *codes,
                               size_t workspace_bytes, w4_stream_t stream);
 
 /*
+ * w4_linear_asym_gidx_noalloc -- w4_linear_asym_gidx for callers that cannot allocate.
+ * The source pages have no counterpart to this call; it exists for host code that may not
+ * allocate device memory when it calls the linear -- for example a program whose framework
+ * owns every device allocation through its own pool, or a serving process that must not call
+ * cudaMalloc after start-up (it synchronizes the device and can fail on a fragmented heap).
+ * Arguments and results are those of w4_linear_asym_gidx without (workspace,
+ * workspace_bytes): the scratch memory lives in one fixed 16 MiB array inside the library,
+ * present on every GPU that loads the library until the process exits.
+ *   - The call allocates nothing (no cudaMalloc / cudaFree, no allocating library routine).
+ *   - Shapes whose scratch (w4_linear_asym_workspace_bytes) exceeds 16 MiB -- M * K bf16
+ *     activations, e.g. M = 2048 at K = 4096 -- return W4_ERR_SHAPE.
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress
+ *     with that device current); make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents (each call overwrites
+ *     what it reads, so nothing needs clearing). Calls that overlap on the GPU -- on
+ *     different streams, or concurrently from several host threads -- race on it.
+ */
+w4_status w4_linear_asym_gidx_noalloc(const void *x, int64_t M, const uint8_t *codes,
+                                      const float *scales, const int8_t *zeros,
+                                      const int32_t *g_idx, const int32_t *perm, int64_t N,
+                                      int64_t K, int64_t n_groups, const float *bias, void *y,
+                                      w4_dtype y_dtype, w4_stream_t stream);
+
+/*
  * w4_validate -- the LoopQ content checks (page "loopq/packed_weight.py", validate) on a
  * device-resident packed weight, reported in the page's order: W4_ERR_VERSION (format not
  * 1 or 2), W4_ERR_SCALE, W4_ERR_HIGH_NIBBLE, W4_ERR_RESERVED_CODE (v1 only). Shape and

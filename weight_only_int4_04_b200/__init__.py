@@ -30,7 +30,7 @@ DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2, torch.float64: 
 
 EXPORTS = (
     "w4_quantize_rtn", "w4_dequantize", "w4_linear", "w4_linear_workspace_bytes", "w4_linear_asym_workspace_bytes",
-    "w4_asym_prepare", "w4_linear_asym_gidx", "w4_validate", "w4_validate_asym",
+    "w4_asym_prepare", "w4_linear_asym_gidx", "w4_linear_asym_gidx_noalloc", "w4_validate", "w4_validate_asym",
     "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
 )
 
@@ -44,6 +44,7 @@ _SIGS = {
     "w4_asym_prepare": [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp],
     "w4_linear_asym_gidx": [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp, _sz,
                             _vp],
+    "w4_linear_asym_gidx_noalloc": [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp],
     "w4_validate": [_vp, _vp, _i64, _i64, _i32, _vp],
     "w4_validate_asym": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
     "w4_device_error": [],
@@ -209,6 +210,26 @@ def linear_asym_gidx(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
     _check(_load().w4_linear_asym_gidx(_ptr(x), M, _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), _ptr(perm),
                                    N, K, G, _ptr(bias), _ptr(out), DTYPES[out.dtype], _ptr(ws), wsb,
                                    _stream()), "w4_linear_asym_gidx")
+    return out
+
+
+def linear_asym_gidx_noalloc(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                             g_idx: torch.Tensor, perm: torch.Tensor | None = None,
+                             bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                             out_dtype=torch.bfloat16) -> torch.Tensor:
+    """``linear_asym_gidx`` through the entry point that allocates no device memory (its
+    scratch is a fixed 16 MiB array inside the library); pass ``out`` to allocate nothing
+    on this side either."""
+    if g_idx.dtype != torch.int32:
+        raise ValueError("g_idx must be int32 here (the conversion would allocate)")
+    _need_cuda(x, codes, scales, zeros, g_idx, perm, bias, out)
+    M, K = x.shape
+    N, G = scales.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check(_load().w4_linear_asym_gidx_noalloc(_ptr(x), M, _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx),
+                                           _ptr(perm), N, K, G, _ptr(bias), _ptr(out), DTYPES[out.dtype],
+                                           _stream()), "w4_linear_asym_gidx_noalloc")
     return out
 
 
