@@ -379,9 +379,9 @@ def main():
                 "steps": e2e_steps,
                 "note": "public Python API per step: pinned-host x -> device, 3 linears, y -> pinned host; "
                         "weights resident in HBM"},
-        "roofline": {"bound": "hbm", "kernel": "gemv_stream_kernel (M=1 decode GEMV)", "achieved": achieved, "peak": hbm_peak,
+        "roofline": {"bound": "hbm", "kernel": "gemv_rows_kernel (M=1 decode GEMV)", "achieved": achieved, "peak": hbm_peak,
                      "unit": "GB/s", "frac": frac, "peak_kind": peak_kind,
-                     "traffic": recorded_traffic("k_gemv.cu", "gemv_decode_m1.md"),
+                     "traffic": recorded_traffic("k_gemv_rows.cu", "gemv_rows_decode_m1.md"),
                      "algorithmic_bytes_per_step": sum(algo_bytes),
                      "launch_us_mean": 1e3 * ms / launches,
                      "per_shape_gbs": {f"{N}x{K}": b / us / 1e3
