@@ -203,6 +203,22 @@ w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8
                            const int32_t *g_idx, int64_t N, int64_t K, int64_t n_groups,
                            w4_stream_t stream);
 
+/*
+ * w4_set_weight_prefetch -- launch policy of the decode linear (process-wide; default 0).
+ * The source pages have no counterpart to this call: it only decides when a kernel starts.
+ * The M = 1 decode kernel is launched with CUDA programmatic dependent launch: it may begin
+ * while the previous kernel of its stream is still running, and it reads x (and bias) and
+ * writes y only after that kernel has completed and its writes are visible. With enable = 1
+ * it also starts streaming codes and scales at once, hiding its ramp-up behind the previous
+ * kernel in a chain of decode linears.
+ * Contract while enabled: the codes and scales of a decode call must already be complete
+ * when the chain of overlapping kernels before it began -- write them earlier and separate
+ * the two by a stream synchronization, an event, or any kernel launched without
+ * programmatic serialization (every other kernel of this library is). Weights written by a
+ * kernel that may still be running may be read stale. Returns the previous setting.
+ */
+int w4_set_weight_prefetch(int enable);
+
 /* Error word written by bounded device-side waits (W4_OK if none expired). Reading it
  * synchronizes the device and clears it. */
 w4_status w4_device_error(void);

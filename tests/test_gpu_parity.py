@@ -255,6 +255,95 @@ def test_linear_zero_rows(w4):
 
 
 # ---------------------------------------------------------------------------
+# decode GEMV (M = 1): TMA stage ring, ragged row blocks and k-tiles, deep rows, launch
+# overlap (programmatic dependent launch with weight prefetch)
+# ---------------------------------------------------------------------------
+
+DECODE_EDGE_NK = [(1, 128), (16, 256), (17, 384), (33, 640), (2368, 2048), (2400, 2432), (4100, 4096),
+                  (5000, 1152), (300, 14336), (64, 28672)]
+
+
+@pytest.mark.parametrize("NK", DECODE_EDGE_NK)
+def test_linear_decode_edges(w4, NK):
+    N, K = NK
+    c = workloads.linear_case(N + 3 * K, 1, N, K, outliers=True)
+    _linear_check(w4, c)
+    _linear_check(w4, c, out_dtype=torch.float32)
+
+
+def test_linear_decode_unaligned_x(w4):
+    """x starting 8 bytes past a 16-byte boundary takes another kernel; same result."""
+    c = workloads.linear_case(77, 1, 300, 2048)
+    codes, scales = oracle_pack(c["W"])
+    buf = torch.zeros(2048 + 8, dtype=torch.bfloat16, device="cuda")
+    buf[4:4 + 2048] = x_dev(c["x_bits"])[0]
+    x = buf[4:4 + 2048].view(1, 2048)
+    assert x.data_ptr() % 16 == 8
+    y = w4.linear(x, dev(codes), dev(scales), 2048, bias=dev(c["bias"]))
+    yr, bound = O.linear(c["x"], codes, scales, 2048, c["bias"])
+    ok, worst = O.check_linear(y_host(y), yr, bound)
+    assert ok, worst
+
+
+def _chain(w4, layers, x0, graph):
+    """y_i = linear(y_{i-1}) for alternating weights on one stream, no host sync between
+    layers; optionally captured once into a CUDA graph and replayed."""
+    outs = [torch.empty((1, layers[i % 2][2].shape[0]), dtype=torch.bfloat16, device="cuda") for i in range(6)]
+
+    def run():
+        x = x0
+        for i in range(6):
+            codes, scales, bias = layers[i % 2][1:]
+            w4.linear(x, codes, scales, x.shape[1], bias=bias, out=outs[i])
+            x = outs[i]
+
+    if graph:
+        run()  # warm-up outside capture (tensor maps, attributes)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run()
+        for o in outs:
+            o.zero_()
+        g.replay()
+        g.replay()
+    else:
+        run()
+    torch.cuda.synchronize()
+    return outs
+
+
+@pytest.mark.parametrize("prefetch", [False, True])
+@pytest.mark.parametrize("graph", [False, True])
+def test_linear_decode_chain_launch_overlap(w4, prefetch, graph):
+    """Each layer reads the previous layer's output: the kernel must not read x (nor write
+    y) before the previous kernel has finished, with and without weight prefetch."""
+    K = 2048
+    layers = []
+    for i in range(2):
+        c = workloads.linear_case(500 + i, 1, K, K)
+        codes, scales = oracle_pack(c["W"])
+        layers.append((c, dev(codes), dev(scales), dev(c["bias"])))
+    torch.cuda.synchronize()
+    prev = w4.set_weight_prefetch(prefetch)
+    try:
+        x0 = x_dev(workloads.linear_case(600, 1, 8, K)["x_bits"])
+        outs = _chain(w4, layers, x0, graph)
+    finally:
+        w4.set_weight_prefetch(prev)
+    x = x0
+    for i, y in enumerate(outs):
+        c = layers[i % 2][0]
+        xb = x.cpu().view(torch.int16).numpy().view(np.uint16)
+        yr, bound = O.linear(O.bf16_bits_to_f32(xb).astype(np.float64), layers[i % 2][1].cpu().numpy(),
+                             layers[i % 2][2].cpu().numpy(), K, c["bias"])
+        ok, worst = O.check_linear(y_host(y), yr, bound)
+        assert ok, (i, worst)
+        x = y
+    assert w4.device_error() == "OK"
+
+
+# ---------------------------------------------------------------------------
 # asymmetric act-order (a6)
 # ---------------------------------------------------------------------------
 

@@ -31,7 +31,7 @@ DTYPES = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2, torch.float64: 
 EXPORTS = (
     "w4_quantize_rtn", "w4_dequantize", "w4_linear", "w4_linear_workspace_bytes", "w4_linear_asym_workspace_bytes",
     "w4_asym_prepare", "w4_linear_asym_gidx", "w4_linear_asym_gidx_noalloc", "w4_validate", "w4_validate_asym",
-    "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
+    "w4_set_weight_prefetch", "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
 )
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -47,6 +47,7 @@ _SIGS = {
     "w4_linear_asym_gidx_noalloc": [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i32, _vp],
     "w4_validate": [_vp, _vp, _i64, _i64, _i32, _vp],
     "w4_validate_asym": [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp],
+    "w4_set_weight_prefetch": [_i32],
     "w4_device_error": [],
     "w4_last_cuda_error": [],
     "w4_status_string": [_i32],
@@ -243,6 +244,13 @@ def validate_asym(codes, scales, zeros, g_idx, K: int) -> str:
     _need_cuda(codes, scales, zeros, g_idx)
     return STATUS[_load().w4_validate_asym(_ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), codes.shape[0], K,
                                        scales.shape[1], _stream())]
+
+
+def set_weight_prefetch(enable: bool) -> bool:
+    """Decode launch policy: stream codes/scales before the previous kernel of the stream
+    has finished (see w4_set_weight_prefetch in include/w4.h for the contract). Returns the
+    previous setting."""
+    return bool(_load().w4_set_weight_prefetch(1 if enable else 0))
 
 
 def device_error() -> str:

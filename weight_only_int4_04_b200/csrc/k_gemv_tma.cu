@@ -1,0 +1,373 @@
+// Decode GEMV (M = 1) on register-fed tensor cores, fed by TMA:
+//   y[n] = sum_k x[k] * (q[n][k] * s[n][k/32]) + b[n]
+//
+// The weight stream (0.625 B per weight) is the whole cost, so the design goal is to keep
+// HBM busy with as few issue slots per weight as possible:
+//   * two CTAs per SM, each owning a balanced contiguous range of 16-row blocks; a single
+//     producer thread walks them in (row block, 2048-column chunk) order and fills a ring of 20 KB
+//     shared-memory stages with 2-D TMA boxes: eight 16-row x 128-byte code boxes and two
+//     16-row x 32-scale boxes, all with the 128-byte swizzle (conflict-free reads below);
+//   * eight consumer warps take one 256-column k-tile of each stage. Per 32-column group a
+//     lane holds one code word of row g and one of row g + 8 (ldmatrix.x4 fetches four such
+//     words, two groups, in one instruction); LOP3 drops each nibble pair into the mantissa
+//     of the bf16 128.0 and one exact bf16x2 FMA removes the offset, which gives the exact
+//     integers q as the A fragment of mma.sync m16n8k16 (bf16 in, fp32 accumulate). The
+//     activations are the B fragment, staged once per CTA in shared memory already in
+//     fragment order. Two MMAs cover a group; the group's fp32 scale multiplies the fp32
+//     group sum in one FFMA per row, so the only rounding besides fp32 accumulation is that
+//     of the scale product -- no bf16 rounding of dequantized weights.
+//     The inner loop is about 1.75 thread-instructions per weight (a CUDA-core dot product
+//     needs ~4.5);
+//   * per row block the warps' partial sums meet in shared memory and are added in a fixed
+//     order (deterministic), the bias is added and y is written.
+// Launch overlap: the kernel is launched with programmatic stream serialization and lets
+// its successor launch at once. It reads x and writes y only after the grid dependency has
+// resolved; when weight prefetch is enabled it streams codes and scales before that, so a
+// chain of decode GEMVs (constant weights) overlaps each kernel's ramp-up with the tail of
+// the previous one. Every wait is bounded (w4_sync.cuh).
+#include <cuda.h>
+
+#include <mutex>
+
+#include "w4_tc.cuh"
+#include "w4_tmap.h"
+
+namespace w4i {
+
+namespace {
+
+constexpr int kWarps = 8;                    // consumer warps; warp kWarps is the producer
+constexpr int kThreads = 32 * (kWarps + 1);  // 288
+constexpr int kRowsPerBlock = 16;            // one m16 MMA tile of weight rows
+constexpr int kKtileCodeBytes = 128;         // 256 columns = 8 groups per k-tile
+constexpr int kKtilesPerStage = kWarps;      // one k-tile per consumer warp per stage
+constexpr int kCodeBox = kRowsPerBlock * kKtileCodeBytes;  // 2 KB
+constexpr int kScaleBox = kRowsPerBlock * 32 * 4;          // 2 KB: 32 scales = 4 k-tiles per row
+constexpr int kStageBytes = kKtilesPerStage * kCodeBox + 2 * kScaleBox;  // 20 KB
+constexpr int kMaxStages = 8;
+constexpr int kRedBytes = 2 * kWarps * kRowsPerBlock * 4;
+constexpr int kBarBytes = 2 * kMaxStages * 8 + 16;
+constexpr int kAlignSlack = 1024;
+// Up to this size two CTAs fit on an SM. Two CTAs of one launch share each SM (16 consumer
+// warps hide more latency than 8); a successor launch's CTAs move in as these exit.
+constexpr int kCoResidentSmem = 112 * 1024;
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxSmem = 227 * 1024;
+constexpr int kBarConsumers = 1;  // named barrier of the consumer warps
+
+struct TmaGemvParams {
+  const __nv_bfloat16 *x;
+  const float *bias;
+  void *y;
+  int64_t N;
+  int64_t K;
+  int64_t NB;    // 16-row blocks
+  int KT;        // 256-column k-tiles per row
+  int SPR;       // stages per row block: ceil(KT / 8)
+  int S;         // stages in the ring
+  int x_bytes;   // permuted activations: KT * 8 groups * 64 bytes
+  int y_dtype;
+  int prefetch;  // stream codes and scales before the grid dependency resolves
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&d)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// D = A * B (+ 0) and D = A * B + D for m16n8k16, bf16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+__device__ __forceinline__ void mma_next(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One code word (columns 8t .. 8t+7 of a group, even column in the low nibble) -> four
+// bf16x2 registers holding the exact signed integers of columns (0,4) (1,5) (2,6) (3,7).
+__device__ __forceinline__ void unpack_signed(uint32_t w, uint32_t (&a)[4]) {
+  a[0] = bf16x2_sub(nib_pair_bf16(w, 0x43084308u), 0x43084308u);
+  a[1] = bf16x2_sub(nib_pair_bf16(w >> 4, 0x43084308u), 0x43084308u);
+  a[2] = bf16x2_sub(nib_pair_bf16(w >> 8, 0x43084308u), 0x43084308u);
+  a[3] = bf16x2_sub(nib_pair_bf16(w >> 12, 0x43084308u), 0x43084308u);
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    gemv_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
+                    const TmaGemvParams p, int32_t *err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte swizzle atoms
+  uint8_t *xs = smem + p.S * kStageBytes;
+  float *red = reinterpret_cast<float *>(xs + p.x_bytes);
+  uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(red) + kRedBytes);
+  uint64_t *empty = full + kMaxStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kMaxStages);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t rb_begin = static_cast<int64_t>(blockIdx.x) * p.NB / gridDim.x;
+  const int64_t rb_end = static_cast<int64_t>(blockIdx.x + 1) * p.NB / gridDim.x;
+  const int total = static_cast<int>(rb_end - rb_begin) * p.SPR;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kWarps);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  grid_launch_dependents();
+
+  if (warp == kWarps) {
+    // ---- producer: one thread issues every TMA box of the CTA's row blocks ----
+    if (lane == 0) {
+      if (!p.prefetch) grid_dependency_wait();
+      int slot = 0, kc = 0;
+      uint32_t phase = 0;
+      int32_t row = static_cast<int32_t>(rb_begin * kRowsPerBlock);
+      for (int i = 0; i < total; ++i) {
+        if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, err)) break;
+        const int kt0 = kc * kKtilesPerStage;
+        const int nkt = (p.KT - kt0) < kKtilesPerStage ? (p.KT - kt0) : kKtilesPerStage;
+        const int nsb = (nkt + 3) / 4;
+        uint8_t *st = smem + slot * kStageBytes;
+        mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox + nsb * kScaleBox));
+        for (int j = 0; j < nkt; ++j)
+          tma_load_2d(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot]);
+        for (int b = 0; b < nsb; ++b)
+          tma_load_2d(st + kKtilesPerStage * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
+                      &full[slot]);
+        if (++kc == p.SPR) {
+          kc = 0;
+          row += kRowsPerBlock;
+        }
+        if (++slot == p.S) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    return;
+  }
+
+  // ---- consumers: x -> shared memory in B-fragment order, once per CTA ----
+  grid_dependency_wait();
+  {
+    const int64_t G = p.K / 32;
+    const uint4 *x4 = reinterpret_cast<const uint4 *>(p.x);
+    for (int c = threadIdx.x; c < p.KT * 32; c += 32 * kWarps) {
+      // c = (group, t): 16 bytes holding columns (8t + e, 8t + e + 4) for e = 0..3
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if ((c >> 2) < G) {
+        const uint4 r = __ldcg(x4 + c);
+        v.x = prmt(r.x, r.z, 0x5410);
+        v.y = prmt(r.x, r.z, 0x7632);
+        v.z = prmt(r.y, r.w, 0x5410);
+        v.w = prmt(r.y, r.w, 0x7632);
+      }
+      reinterpret_cast<uint4 *>(xs)[c] = v;
+    }
+  }
+  named_barrier_sync(kBarConsumers, 32 * kWarps);
+
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t stages0 = smem_u32(smem);
+  // ldmatrix.x4: lanes 8i .. 8i+7 address the rows of matrix i = (rows 0-7 | rows 8-15) x
+  // (group 2p | group 2p+1); the 128-byte swizzle puts 16-byte chunk c of row r at c ^ (r & 7).
+  const uint32_t ld_row = static_cast<uint32_t>(((lane & 7) + ((lane >> 3) & 1) * 8) * kKtileCodeBytes);
+  const uint32_t ld_xor = static_cast<uint32_t>(lane & 7), ld_hi = static_cast<uint32_t>(lane >> 4);
+  // this warp's 8 scales per row: chunks 2(w%4), 2(w%4)+1 of scale box w/4
+  const uint32_t sbox = static_cast<uint32_t>(kKtilesPerStage * kCodeBox + (warp >> 2) * kScaleBox);
+  const uint32_t sch = static_cast<uint32_t>(2 * (warp & 3));
+  const uint32_t s_lo = static_cast<uint32_t>(g * 128) + ((sch ^ g) << 4);
+  const uint32_t s_hi = static_cast<uint32_t>(g * 128) + (((sch + 1) ^ g) << 4);
+
+  float acc0 = 0.0f, acc1 = 0.0f;  // rows g and g + 8 of the current row block
+  int buf = 0, slot = 0, kc = 0;
+  uint32_t phase = 0;
+  int64_t row0 = rb_begin * kRowsPerBlock;
+  for (int i = 0; i < total; ++i) {
+    mbar_wait(&full[slot], phase, abort_flag, err);
+    const int kt = kc * kKtilesPerStage + warp;
+    if (kt < p.KT) {
+      const uint32_t st = stages0 + static_cast<uint32_t>(slot * kStageBytes);
+      const uint32_t cb = st + static_cast<uint32_t>(warp * kCodeBox) + ld_row;
+      uint32_t w[4][4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ldsm_x4(cb + ((((2u * q) + ld_hi) ^ ld_xor) << 4), w[q]);
+      const uint8_t *sp = smem + slot * kStageBytes + sbox;
+      const uint4 sg0 = *reinterpret_cast<const uint4 *>(sp + s_lo);
+      const uint4 sg1 = *reinterpret_cast<const uint4 *>(sp + s_hi);
+      const uint4 sh0 = *reinterpret_cast<const uint4 *>(sp + 1024 + s_lo);
+      const uint4 sh1 = *reinterpret_cast<const uint4 *>(sp + 1024 + s_hi);
+      const float s0[8] = {__uint_as_float(sg0.x), __uint_as_float(sg0.y), __uint_as_float(sg0.z),
+                           __uint_as_float(sg0.w), __uint_as_float(sg1.x), __uint_as_float(sg1.y),
+                           __uint_as_float(sg1.z), __uint_as_float(sg1.w)};
+      const float s1[8] = {__uint_as_float(sh0.x), __uint_as_float(sh0.y), __uint_as_float(sh0.z),
+                           __uint_as_float(sh0.w), __uint_as_float(sh1.x), __uint_as_float(sh1.y),
+                           __uint_as_float(sh1.z), __uint_as_float(sh1.w)};
+      const uint4 *xk = reinterpret_cast<const uint4 *>(xs) + kt * 32 + t;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint4 xf = xk[4 * j];
+        uint32_t a[4], b[4];
+        unpack_signed(w[j >> 1][(j & 1) * 2], a);      // row g
+        unpack_signed(w[j >> 1][(j & 1) * 2 + 1], b);  // row g + 8
+        float d[4];
+        mma_first(d, a[0], b[0], a[1], b[1], xf.x, xf.y);
+        mma_next(d, a[2], b[2], a[3], b[3], xf.z, xf.w);
+        acc0 = fmaf(d[0], s0[j], acc0);
+        acc1 = fmaf(d[2], s1[j], acc1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    if (++slot == p.S) {
+      slot = 0;
+      phase ^= 1u;
+    }
+
+    if (++kc == p.SPR) {
+      // row block complete: the eight warps' sums meet in shared memory (fixed order)
+      kc = 0;
+      float *r = red + buf * (kWarps * kRowsPerBlock);
+      if (t == 0) {
+        r[warp * kRowsPerBlock + g] = acc0;
+        r[warp * kRowsPerBlock + g + 8] = acc1;
+      }
+      named_barrier_sync(kBarConsumers, 32 * kWarps);
+      if (warp == static_cast<int>((row0 / kRowsPerBlock) % kWarps) && lane < kRowsPerBlock) {
+        const int64_t n = row0 + lane;
+        if (n < p.N) {
+          float v = 0.0f;
+#pragma unroll
+          for (int w2 = 0; w2 < kWarps; ++w2) v += r[w2 * kRowsPerBlock + lane];
+          if (p.bias) v += __ldcg(p.bias + n);
+          if (p.y_dtype == W4_F32)
+            static_cast<float *>(p.y)[n] = v;
+          else
+            static_cast<__nv_bfloat16 *>(p.y)[n] = __float2bfloat16_rn(v);
+        }
+      }
+      acc0 = 0.0f;
+      acc1 = 0.0f;
+      buf ^= 1;  // the next block writes the other buffer; two barriers apart from this read
+      row0 += kRowsPerBlock;
+    }
+  }
+}
+
+int sm_count_current() {
+  static int counts[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem) {
+  if (lp.M != 1 || lp.asym) return false;
+  if (lp.K % 128 != 0 || lp.N > 0x7fffffffLL) return false;  // TMA: 16-byte row strides, int32 rows
+  if (lp.y_dtype != W4_BF16 && lp.y_dtype != W4_F32) return false;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(lp.codes) | reinterpret_cast<uintptr_t>(lp.scales) |
+                      reinterpret_cast<uintptr_t>(lp.x);
+  if (a % 16 != 0) return false;
+  const int64_t KT = (lp.K + 255) / 256;
+  const int64_t x_bytes = KT * 512;
+  const int64_t fixed = kAlignSlack + x_bytes + kRedBytes + kBarBytes;
+  int64_t S = (kCoResidentSmem - fixed) / kStageBytes;
+  if (S < 4) S = (kMaxSmem - fixed) / kStageBytes;  // long rows: give up co-residency for depth
+  if (S > kMaxStages) S = kMaxStages;
+  if (S < 2) return false;
+  q->x = lp.x;
+  q->bias = lp.bias;
+  q->y = lp.y;
+  q->N = lp.N;
+  q->K = lp.K;
+  q->NB = (lp.N + kRowsPerBlock - 1) / kRowsPerBlock;
+  q->KT = static_cast<int>(KT);
+  q->SPR = static_cast<int>((KT + kKtilesPerStage - 1) / kKtilesPerStage);
+  q->S = static_cast<int>(S);
+  q->x_bytes = static_cast<int>(x_bytes);
+  q->y_dtype = lp.y_dtype;
+  q->prefetch = 0;
+  *smem = static_cast<int>(fixed + S * kStageBytes);
+  return true;
+}
+
+cudaError_t ensure_smem_attr() {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(gemv_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+bool gemv_tma_supports(const LinearParams &p) {
+  TmaGemvParams q;
+  int smem;
+  return make_params(p, &q, &smem) && encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, int32_t *err, cudaStream_t stream) {
+  TmaGemvParams q;
+  int smem = 0;
+  if (!make_params(lp, &q, &smem)) return cudaErrorNotSupported;
+  q.prefetch = prefetch ? 1 : 0;
+  const int64_t P = lp.K / 2, G = lp.K / 32;
+  CUtensorMap mc, ms;
+  if (!make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes, kRowsPerBlock,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, G, lp.N, G * 4, 32, kRowsPerBlock,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  cudaError_t e = ensure_smem_attr();
+  if (e != cudaSuccess) return e;
+  const int64_t slots = static_cast<int64_t>(sm_count_current()) * kCtasPerSm;
+  int64_t grid = q.NB < slots ? q.NB : slots;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_tma_kernel, mc, ms, q, err);
+}
+
+}  // namespace w4i

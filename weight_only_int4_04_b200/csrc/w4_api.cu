@@ -2,6 +2,7 @@
 // selection and error reporting. No device memory is allocated here; the only device state
 // is the static status words below (one per loaded library, shared by every call).
 #include <algorithm>
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <vector>
@@ -38,6 +39,10 @@ w4_status symbol_ptr(T **out, const T &sym) {
   return W4_OK;
 }
 
+// Decode launch policy (w4_set_weight_prefetch): stream codes and scales before the
+// previous kernel of the stream has finished.
+std::atomic<int> g_weight_prefetch{0};
+
 // Tensor-core GEMM is used above this M (and whenever the decode kernels do not apply).
 constexpr int64_t kTcMinM = 17;
 
@@ -51,19 +56,23 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
   int32_t *err = nullptr;
   const w4_status st = symbol_ptr(&err, g_device_error);
   if (st != W4_OK) return st;
-  // M dispatch: M = 1 -> the register-streaming GEMV; M <= 16 -> the tensor-core decode
-  // kernel (bulk-copy slot ring, mma.sync); larger M -> the tcgen05 GEMM; the other GEMV
-  // kernels and the generic kernel take the shapes the fast paths cannot (unaligned rows,
-  // odd widths, unsorted act-order maps). W4_GEMV=stream|mma picks the alternative M = 1
-  // kernels (for comparisons only).
+  // M dispatch: M = 1 -> the TMA-fed tensor-core GEMV (symmetric codes, K a multiple of
+  // 128), else the register-streaming GEMV; M <= 16 -> the tensor-core decode kernel
+  // (bulk-copy slot ring, mma.sync); larger M -> the tcgen05 GEMM; the other GEMV kernels and
+  // the generic kernel take the shapes the fast paths cannot (unaligned rows, odd widths,
+  // unsorted act-order maps). W4_GEMV=rows|stream|mma picks an alternative M = 1 kernel (for
+  // comparisons only).
   static const int m1_kernel = [] {
     const char *v = getenv("W4_GEMV");
     if (v != nullptr && strcmp(v, "stream") == 0) return 1;
     if (v != nullptr && strcmp(v, "mma") == 0) return 2;
+    if (v != nullptr && strcmp(v, "rows") == 0) return 3;
     return 0;
   }();
   cudaError_t e;
-  if (m1_kernel == 0 && w4i::gemv_rows_supports(p)) {
+  if (m1_kernel == 0 && w4i::gemv_tma_supports(p)) {
+    e = w4i::launch_gemv_tma(p, g_weight_prefetch.load(std::memory_order_relaxed) != 0, err, stream);
+  } else if ((m1_kernel == 0 || m1_kernel == 3) && w4i::gemv_rows_supports(p)) {
     e = w4i::launch_gemv_rows(p, stream);
   } else if (m1_kernel != 2 && w4i::gemv_stream_supports(p)) {
     e = w4i::launch_gemv_stream(p, err, stream);
@@ -277,6 +286,10 @@ w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8
   if (f & w4i::FLAG_ZERO) return W4_ERR_ZERO;
   if (f & w4i::FLAG_GIDX) return W4_ERR_GIDX;
   return W4_OK;
+}
+
+int w4_set_weight_prefetch(int enable) {
+  return g_weight_prefetch.exchange(enable != 0 ? 1 : 0);
 }
 
 w4_status w4_device_error(void) {

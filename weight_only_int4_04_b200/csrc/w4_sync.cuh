@@ -101,4 +101,16 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization
+// may start while the previous kernel of its stream is still running; grid_dependency_wait
+// blocks the calling thread until that kernel has completed and its memory writes are
+// visible (it returns at once when there is no such dependency).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allows the next kernel of the stream (if launched with programmatic serialization) to be
+// scheduled once every CTA of this grid has executed this or exited.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace w4i
