@@ -54,6 +54,7 @@ constexpr int kCoResidentSmem = 112 * 1024;
 constexpr int kCtasPerSm = 2;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kBarConsumers = 1;  // named barrier of the consumer warps
+constexpr int kXBatch = 8;        // x chunks in flight per consumer thread (K <= 16384 in one batch)
 
 struct TmaGemvParams {
   const __nv_bfloat16 *x;
@@ -62,6 +63,7 @@ struct TmaGemvParams {
   int64_t N;
   int64_t K;
   int64_t NB;    // 16-row blocks
+  int rb_q, rb_r; // CTA c owns rb_q + (c < rb_r) row blocks starting at c * rb_q + min(c, rb_r)
   int KT;        // 256-column k-tiles per row
   int SPR;       // stages per row block: ceil(KT / 8)
   int S;         // stages in the ring
@@ -121,9 +123,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kMaxStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t rb_begin = static_cast<int64_t>(blockIdx.x) * p.NB / gridDim.x;
-  const int64_t rb_end = static_cast<int64_t>(blockIdx.x + 1) * p.NB / gridDim.x;
-  const int total = static_cast<int>(rb_end - rb_begin) * p.SPR;
+  const int cta = static_cast<int>(blockIdx.x);
+  const int64_t rb_begin = static_cast<int64_t>(cta) * p.rb_q + (cta < p.rb_r ? cta : p.rb_r);
+  const int total = (p.rb_q + (cta < p.rb_r ? 1 : 0)) * p.SPR;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.S; ++i) {
@@ -171,19 +173,30 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ---- consumers: x -> shared memory in B-fragment order, once per CTA ----
   grid_dependency_wait();
   {
-    const int64_t G = p.K / 32;
+    // all loads of a thread are issued before any is used: one memory round trip, not one
+    // per chunk. Chunk c = (group, t) holds columns (8t + e, 8t + e + 4) for e = 0..3.
+    const int G = static_cast<int>(p.K / 32);
+    const int chunks = p.KT * 32;
     const uint4 *x4 = reinterpret_cast<const uint4 *>(p.x);
-    for (int c = threadIdx.x; c < p.KT * 32; c += 32 * kWarps) {
-      // c = (group, t): 16 bytes holding columns (8t + e, 8t + e + 4) for e = 0..3
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if ((c >> 2) < G) {
-        const uint4 r = __ldcg(x4 + c);
-        v.x = prmt(r.x, r.z, 0x5410);
-        v.y = prmt(r.x, r.z, 0x7632);
-        v.z = prmt(r.y, r.w, 0x5410);
-        v.w = prmt(r.y, r.w, 0x7632);
+    for (int base = static_cast<int>(threadIdx.x); base < chunks; base += kXBatch * 32 * kWarps) {
+      uint4 r4[kXBatch];
+#pragma unroll
+      for (int k = 0; k < kXBatch; ++k) {
+        const int c = base + k * 32 * kWarps;
+        r4[k] = (c < chunks && (c >> 2) < G) ? __ldcg(x4 + c) : make_uint4(0u, 0u, 0u, 0u);
       }
-      reinterpret_cast<uint4 *>(xs)[c] = v;
+#pragma unroll
+      for (int k = 0; k < kXBatch; ++k) {
+        const int c = base + k * 32 * kWarps;
+        if (c < chunks) {
+          uint4 v;
+          v.x = prmt(r4[k].x, r4[k].z, 0x5410);
+          v.y = prmt(r4[k].x, r4[k].z, 0x7632);
+          v.z = prmt(r4[k].y, r4[k].w, 0x5410);
+          v.w = prmt(r4[k].y, r4[k].w, 0x7632);
+          reinterpret_cast<uint4 *>(xs)[c] = v;
+        }
+      }
     }
   }
   named_barrier_sync(kBarConsumers, 32 * kWarps);
@@ -200,8 +213,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t s_lo = static_cast<uint32_t>(g * 128) + ((sch ^ g) << 4);
   const uint32_t s_hi = static_cast<uint32_t>(g * 128) + (((sch + 1) ^ g) << 4);
 
+  uint32_t ld_off[4];  // this lane's four swizzled ldmatrix offsets (q: groups 2q, 2q + 1)
+#pragma unroll
+  for (int q = 0; q < 4; ++q) ld_off[q] = ld_row + ((((2u * q) + ld_hi) ^ ld_xor) << 4);
+
   float acc0 = 0.0f, acc1 = 0.0f;  // rows g and g + 8 of the current row block
-  int buf = 0, slot = 0, kc = 0;
+  int buf = 0, slot = 0, kc = 0, rbl = 0;
   uint32_t phase = 0;
   int64_t row0 = rb_begin * kRowsPerBlock;
   for (int i = 0; i < total; ++i) {
@@ -209,10 +226,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int kt = kc * kKtilesPerStage + warp;
     if (kt < p.KT) {
       const uint32_t st = stages0 + static_cast<uint32_t>(slot * kStageBytes);
-      const uint32_t cb = st + static_cast<uint32_t>(warp * kCodeBox) + ld_row;
+      const uint32_t cb = st + static_cast<uint32_t>(warp * kCodeBox);
       uint32_t w[4][4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) ldsm_x4(cb + ((((2u * q) + ld_hi) ^ ld_xor) << 4), w[q]);
+      for (int q = 0; q < 4; ++q) ldsm_x4(cb + ld_off[q], w[q]);
       const uint8_t *sp = smem + slot * kStageBytes + sbox;
       const uint4 sg0 = *reinterpret_cast<const uint4 *>(sp + s_lo);
       const uint4 sg1 = *reinterpret_cast<const uint4 *>(sp + s_hi);
@@ -254,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         r[warp * kRowsPerBlock + g + 8] = acc1;
       }
       named_barrier_sync(kBarConsumers, 32 * kWarps);
-      if (warp == static_cast<int>((row0 / kRowsPerBlock) % kWarps) && lane < kRowsPerBlock) {
+      if (warp == (rbl & (kWarps - 1)) && lane < kRowsPerBlock) {
         const int64_t n = row0 + lane;
         if (n < p.N) {
           float v = 0.0f;
@@ -271,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       acc1 = 0.0f;
       buf ^= 1;  // the next block writes the other buffer; two barriers apart from this read
       row0 += kRowsPerBlock;
+      ++rbl;
     }
   }
 }
@@ -307,6 +325,7 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem) {
   q->N = lp.N;
   q->K = lp.K;
   q->NB = (lp.N + kRowsPerBlock - 1) / kRowsPerBlock;
+  if (q->NB >= (int64_t(1) << 31) / 64) return false;
   q->KT = static_cast<int>(KT);
   q->SPR = static_cast<int>((KT + kKtilesPerStage - 1) / kKtilesPerStage);
   q->S = static_cast<int>(S);
@@ -356,7 +375,9 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, int32_t *err,
   cudaError_t e = ensure_smem_attr();
   if (e != cudaSuccess) return e;
   const int64_t slots = static_cast<int64_t>(sm_count_current()) * kCtasPerSm;
-  int64_t grid = q.NB < slots ? q.NB : slots;
+  const int64_t grid = q.NB < slots ? q.NB : slots;
+  q.rb_q = static_cast<int>(q.NB / grid);
+  q.rb_r = static_cast<int>(q.NB % grid);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);

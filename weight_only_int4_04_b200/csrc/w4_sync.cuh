@@ -74,9 +74,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
                                           int32_t *err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
-    __nanosleep(64);  // back off: a spinning waiter would take issue slots from the math warps
+  for (uint32_t n = 0;; ++n) {
+    // The hint lets the hardware suspend the thread until the phase completes (it wakes on
+    // completion, not on a timer), so a waiter takes no issue slots and resumes at once.
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (n >= 32) __nanosleep(256);  // only if the suspend keeps returning early
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
