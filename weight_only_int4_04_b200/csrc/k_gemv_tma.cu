@@ -70,6 +70,7 @@ struct TmaGemvParams {
   int x_bytes;   // permuted activations: KT * 8 groups * 64 bytes
   int y_dtype;
   int prefetch;  // stream codes and scales before the grid dependency resolves
+  int boxes3d;   // 1: one 3-D box per stage for the codes and one for the scales
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&d)[4]) {
@@ -151,12 +152,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int nkt = (p.KT - kt0) < kKtilesPerStage ? (p.KT - kt0) : kKtilesPerStage;
         const int nsb = (nkt + 3) / 4;
         uint8_t *st = smem + slot * kStageBytes;
-        mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox + nsb * kScaleBox));
-        for (int j = 0; j < nkt; ++j)
-          tma_load_2d(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot]);
-        for (int b = 0; b < nsb; ++b)
-          tma_load_2d(st + kKtilesPerStage * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
-                      &full[slot]);
+        if (p.boxes3d) {
+          // whole-stage boxes; k-tiles past the row end read as zeros (and count as bytes)
+          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(kStageBytes));
+          tma_load_3d(st, &tm_codes, 0, row, kt0, &full[slot]);
+          tma_load_3d(st + kKtilesPerStage * kCodeBox, &tm_scales, 0, row, kt0 / 4, &full[slot]);
+        } else {
+          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox + nsb * kScaleBox));
+          for (int j = 0; j < nkt; ++j)
+            tma_load_2d(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot]);
+          for (int b = 0; b < nsb; ++b)
+            tma_load_2d(st + kKtilesPerStage * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
+                        &full[slot]);
+        }
         if (++kc == p.SPR) {
           kc = 0;
           row += kRowsPerBlock;
@@ -367,10 +375,19 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, int32_t *err,
   q.prefetch = prefetch ? 1 : 0;
   const int64_t P = lp.K / 2, G = lp.K / 32;
   CUtensorMap mc, ms;
-  if (!make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes, kRowsPerBlock,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, G, lp.N, G * 4, 32, kRowsPerBlock,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+  // 3-D boxes need whole 256-column tiles of codes and whole 1024-column quads of scales in
+  // every row (a box never reaches past a row's end into the next row)
+  q.boxes3d = lp.K % 1024 == 0 &&
+              make_map_3d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, kKtileCodeBytes, lp.N, P / kKtileCodeBytes,
+                          P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, kKtilesPerStage,
+                          CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map_3d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, 32, lp.N, G / 32, G * 4, 128, 32,
+                          kRowsPerBlock, kKtilesPerStage / 4, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!q.boxes3d &&
+      (!make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes, kRowsPerBlock,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+       !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, G, lp.N, G * 4, 32, kRowsPerBlock,
+                    CU_TENSOR_MAP_SWIZZLE_128B)))
     return cudaErrorInvalidValue;
   cudaError_t e = ensure_smem_attr();
   if (e != cudaSuccess) return e;

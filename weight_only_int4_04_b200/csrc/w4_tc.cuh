@@ -20,6 +20,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst_smem, const void *tmap, in
       : "memory");
 }
 
+// 3-D TMA load of one box; coordinates innermost first.
+__device__ __forceinline__ void tma_load_3d(void *dst_smem, const void *tmap, int32_t x, int32_t y, int32_t z,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand in the 128-byte swizzled canonical
 // layout: rows of 128 bytes (64 bf16), 8-row groups 1024 bytes apart, 16-byte chunks XORed
 // with the row index inside the group. Fields: start address >> 4 in bits [0,14), leading

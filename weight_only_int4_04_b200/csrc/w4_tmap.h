@@ -39,4 +39,20 @@ inline bool make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *ba
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Three-dimensional view {inner, outer, tiles} of a row-major array: element (i, r, j) is at
+// byte r * row_bytes + j * tile_bytes + i * element size. Used to fetch several consecutive
+// column tiles of a block of rows in one box ({box_inner, box_outer, box_tiles}).
+inline bool make_map_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                        uint64_t outer, uint64_t tiles, uint64_t row_bytes, uint64_t tile_bytes,
+                        uint32_t box_inner, uint32_t box_outer, uint32_t box_tiles, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {inner, outer, tiles};
+  const cuuint64_t strides[2] = {row_bytes, tile_bytes};
+  const cuuint32_t box[3] = {box_inner, box_outer, box_tiles};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace w4i
