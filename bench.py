@@ -399,8 +399,9 @@ def main():
 
 
 def detail_workloads(w4, dev, hbm_peak, tc_peak):
-    """Named workloads of the other configurations. Each entry builds its inputs and
-    returns (call, report) where report(us) gives the line's figures."""
+    """Named workloads of the other configurations. Each entry builds its inputs and returns
+    (calls, report): calls cycle through ROTATE weight copies (so that no launch finds its
+    weights in L2) and report(us) gives the line's figures."""
     import torch
 
     def bf16(bits):
@@ -410,18 +411,21 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
         N, K = workloads.ODD_DEQUANT_SHAPE
         c = workloads.decode_case(N, K)
         codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
+        copies = [(codes.clone(), scales.clone()) for _ in range(ROTATE)]
         o = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
         nb = payload(N, K) + 2 * N * K
-        return (lambda: w4.dequantize(codes, scales, K, torch.bfloat16, out=o),
+        return ([lambda c=c, s=s: w4.dequantize(c, s, K, torch.bfloat16, out=o) for c, s in copies],
                 lambda us: {"us": us, "gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
 
     def quantize():
         N, K = workloads.BATCHED_SHAPE
         c = workloads.decode_case(N, K, M=1, config=3, bias=True)
-        W = torch.from_numpy(c["W"]).to(dev)
+        W = torch.from_numpy(c["W"]).to(dev)  # 235 MB of fp32 input: larger than L2 by itself
         st = torch.zeros(1, dtype=torch.int32, device=dev)
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((N, K // 32), dtype=torch.float32, device=dev)
         nb = 4 * N * K + payload(N, K)
-        return (lambda: w4.quantize_rtn(W, status=st),
+        return ([lambda: w4.quantize_rtn(W, status=st, out=(codes, scales))],
                 lambda us: {"us": us, "gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
 
     def batched(M):
@@ -429,11 +433,12 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
             N, K = workloads.BATCHED_SHAPE
             c = workloads.decode_case(N, K, M=M, config=3, bias=True)
             codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
+            copies = [(codes.clone(), scales.clone()) for _ in range(ROTATE)]
             bias = torch.from_numpy(c["bias"]).to(dev)
             x = bf16(c["x_bits"])
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             fl = 2.0 * M * N * K
-            return (lambda: w4.linear(x, codes, scales, K, bias=bias, out=y),
+            return ([lambda c=c, s=s: w4.linear(x, c, s, K, bias=bias, out=y) for c, s in copies],
                     lambda us: {"us": us, "weight_gbs": payload(N, K) / us / 1e3,
                                 "frac_hbm": payload(N, K) / us / 1e3 / hbm_peak, "tflops": fl / us / 1e6})
         return make
@@ -445,7 +450,7 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
             x = bf16(c["x_bits"])
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             fl = 2.0 * M * N * K
-            return (lambda: w4.linear(x, codes, scales, K, out=y),
+            return ([lambda: w4.linear(x, codes, scales, K, out=y)],
                     lambda us: {"us": us, "tflops": fl / us / 1e6, "frac_tensor": fl / us / 1e6 / tc_peak})
         return make
 
@@ -456,12 +461,16 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
             sc, perm = w4.asym_prepare(torch.from_numpy(a["codes"]).to(dev), gi, a["K"], a["n_groups"])
             s = torch.from_numpy(a["scales"]).to(dev)
             z = torch.from_numpy(a["zeros"]).to(dev)
+            copies = [(sc.clone(), s.clone(), z.clone()) for _ in range(ROTATE)]
             x = bf16(a["x_bits"])
             b = torch.from_numpy(a["bias"]).to(dev)
             y = torch.empty((M, a["N"]), dtype=torch.bfloat16, device=dev)
+            need = w4.asym_workspace_bytes(M, a["N"], a["K"], a["n_groups"])
+            ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
             nb = a["codes"].size + 4 * a["scales"].size + a["zeros"].size + 4 * a["K"]
             fl = 2.0 * M * a["N"] * a["K"]
-            return (lambda: w4.linear_asym_gidx(x, sc, s, z, gi, perm=perm, bias=b, out=y),
+            return ([lambda c=c, s_=s_, z_=z_: w4.linear_asym_gidx(x, c, s_, z_, gi, perm=perm, bias=b, out=y,
+                                                                   workspace=ws) for c, s_, z_ in copies],
                     lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak,
                                 "tflops": fl / us / 1e6})
         return make
@@ -477,38 +486,36 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
 
 
 def run_detail(w4, dev, hbm_peak, tc_peak, only=None, iters=None, warmup=2):
-    """Time each named workload with CUDA events per call and a 256 MiB L2 flush between
-    calls (outside the timed events); report the median call."""
+    """Time each named workload the way the headline is timed: a CUDA graph of back-to-back
+    calls cycling through rotating weight copies, CUDA events around one replay; the time per
+    call is the replay time divided by the calls."""
     import torch
 
-    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
     out = {}
+    side = torch.cuda.Stream()
     for name, make in detail_workloads(w4, dev, hbm_peak, tc_peak).items():
         if only is not None and name != only:
             continue
-        call, report = make()
-        n = iters if iters is not None else (5 if name.startswith("prefill") else 20)
-        for _ in range(warmup):
-            call()
-        out[name] = report(1e3 * time_calls(call, n, flush))
-        del call
-        torch.cuda.empty_cache()
-    return out
-
-
-def time_calls(fn, iters, flush):
-    import torch
-    ts = []
-    for _ in range(iters):
-        flush.zero_()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
+        calls, report = make()
+        reps = iters if iters is not None else (10 if name.startswith("prefill") else 100)
+        for i in range(max(warmup, len(calls))):
+            calls[i % len(calls)]()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(reps):
+                calls[i % len(calls)]()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        fn()
+        g.replay()
         b.record()
         torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
-    return float(np.median(ts))
+        out[name] = report(1e3 * a.elapsed_time(b) / reps)
+        del g, calls
+        torch.cuda.empty_cache()
+    return out
 
 
 if __name__ == "__main__":

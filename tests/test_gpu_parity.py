@@ -271,6 +271,17 @@ def test_linear_decode_edges(w4, NK):
     _linear_check(w4, c, out_dtype=torch.float32)
 
 
+@pytest.mark.parametrize("M", [2, 3, 7, 8, 9, 13, 16])
+@pytest.mark.parametrize("NK", [(2400, 2432), (300, 14336), (33, 1152)])
+def test_linear_small_m_tensor_core_path(w4, M, NK):
+    """Small M on the TMA-fed tensor-core kernel (activation rows as MMA columns): ragged
+    row blocks and k-tiles, one and two n-tiles, activations up to shared-memory size."""
+    N, K = NK
+    c = workloads.linear_case(M * 31 + N + K, M, N, K, outliers=True)
+    _linear_check(w4, c)
+    _linear_check(w4, c, out_dtype=torch.float32)
+
+
 def test_linear_decode_unaligned_x(w4):
     """x starting 8 bytes past a 16-byte boundary takes another kernel; same result."""
     c = workloads.linear_case(77, 1, 300, 2048)

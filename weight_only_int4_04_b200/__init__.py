@@ -113,18 +113,26 @@ def _need_cuda(*ts):
             raise ValueError("w4: tensors must be contiguous CUDA tensors (no CPU fallback)")
 
 
-def quantize_rtn(W: torch.Tensor, status: torch.Tensor | None = None):
+def quantize_rtn(W: torch.Tensor, status: torch.Tensor | None = None, out=None):
     """RTN symmetric group-32 quantization of fp32 ``W [N, K]`` -> ``(codes, scales)``.
 
     With ``status`` (an int32 CUDA tensor of one element, zeroed by the caller) the call
     stays asynchronous and a non-finite W sets it to the NONFINITE code; without it the
-    call synchronizes and raises ``W4Error`` for a non-finite W."""
+    call synchronizes and raises ``W4Error`` for a non-finite W. ``out``: optional
+    preallocated ``(codes uint8 [N, ceil(K/2)], scales float32 [N, ceil(K/32)])``."""
     _need_cuda(W, status)
     if W.dtype != torch.float32 or W.dim() != 2:
         raise ValueError("W must be a 2-D float32 tensor")
     N, K = W.shape
-    codes = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=W.device)
-    scales = torch.empty((N, (K + 31) // 32), dtype=torch.float32, device=W.device)
+    if out is None:
+        codes = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=W.device)
+        scales = torch.empty((N, (K + 31) // 32), dtype=torch.float32, device=W.device)
+    else:
+        codes, scales = out
+        _need_cuda(codes, scales)
+        if codes.shape != (N, (K + 1) // 2) or scales.shape != (N, (K + 31) // 32) or \
+                codes.dtype != torch.uint8 or scales.dtype != torch.float32:
+            raise ValueError("out must be (uint8 [N, ceil(K/2)], float32 [N, ceil(K/32)])")
     _check(_load().w4_quantize_rtn(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(status), _stream()),
            "w4_quantize_rtn")
     return codes, scales

@@ -1,23 +1,25 @@
-// Decode GEMV (M = 1) on register-fed tensor cores, fed by TMA:
-//   y[n] = sum_k x[k] * (q[n][k] * s[n][k/32]) + b[n]
+// Decode GEMV / small-M linear (M <= 16) on register-fed tensor cores, fed by TMA:
+//   y[m][n] = sum_k x[m][k] * (q[n][k] * s[n][k/32]) + b[n]
 //
 // The weight stream (0.625 B per weight) is the whole cost, so the design goal is to keep
 // HBM busy with as few issue slots per weight as possible:
-//   * two CTAs per SM, each owning a balanced contiguous range of 16-row blocks; a single
-//     producer thread walks them in (row block, 2048-column chunk) order and fills a ring of 20 KB
-//     shared-memory stages with 2-D TMA boxes: eight 16-row x 128-byte code boxes and two
-//     16-row x 32-scale boxes, all with the 128-byte swizzle (conflict-free reads below);
+//   * one or two CTAs per SM (two when their shared memory fits), each owning a balanced
+//     contiguous range of 16-row blocks; a single producer thread walks them in (row block,
+//     2048-column chunk) order and fills a ring of 20 KB shared-memory stages with TMA boxes
+//     of codes and scales, all with the 128-byte swizzle (conflict-free reads below);
 //   * eight consumer warps take one 256-column k-tile of each stage. Per 32-column group a
 //     lane holds one code word of row g and one of row g + 8 (ldmatrix.x4 fetches four such
 //     words, two groups, in one instruction); LOP3 drops each nibble pair into the mantissa
 //     of the bf16 128.0 and one exact bf16x2 FMA removes the offset, which gives the exact
 //     integers q as the A fragment of mma.sync m16n8k16 (bf16 in, fp32 accumulate). The
-//     activations are the B fragment, staged once per CTA in shared memory already in
-//     fragment order. Two MMAs cover a group; the group's fp32 scale multiplies the fp32
-//     group sum in one FFMA per row, so the only rounding besides fp32 accumulation is that
-//     of the scale product -- no bf16 rounding of dequantized weights.
-//     The inner loop is about 1.75 thread-instructions per weight (a CUDA-core dot product
-//     needs ~4.5);
+//     activations are the B fragment: with M = 1 every MMA column carries x (broadcast),
+//     otherwise column n of n-tile j carries activation row 8j + n. Two MMAs cover a group;
+//     the group's fp32 scale multiplies the fp32 group sum in one FFMA per accumulator, so
+//     the only rounding besides fp32 accumulation is that of the scale product -- no bf16
+//     rounding of dequantized weights. At M = 1 the inner loop is about 1.75
+//     thread-instructions per weight (a CUDA-core dot product needs ~4.5);
+//   * x arrives by one bulk copy per activation row, issued as soon as the grid dependency
+//     resolves, and is permuted in place (within each 16-byte chunk) into fragment order;
 //   * per row block the warps' partial sums meet in shared memory and are added in a fixed
 //     order (deterministic), the bias is added and y is written.
 // Launch overlap: the kernel is launched with programmatic stream serialization and lets
@@ -45,16 +47,15 @@ constexpr int kCodeBox = kRowsPerBlock * kKtileCodeBytes;  // 2 KB
 constexpr int kScaleBox = kRowsPerBlock * 32 * 4;          // 2 KB: 32 scales = 4 k-tiles per row
 constexpr int kStageBytes = kKtilesPerStage * kCodeBox + 2 * kScaleBox;  // 20 KB
 constexpr int kMaxStages = 8;
-constexpr int kRedBytes = 2 * kWarps * kRowsPerBlock * 4;
-constexpr int kBarBytes = 2 * kMaxStages * 8 + 16;
+constexpr int kBarBytes = (2 * kMaxStages + 1) * 8 + 16;
 constexpr int kAlignSlack = 1024;
-// Up to this size two CTAs fit on an SM. Two CTAs of one launch share each SM (16 consumer
-// warps hide more latency than 8); a successor launch's CTAs move in as these exit.
-constexpr int kCoResidentSmem = 112 * 1024;
-constexpr int kCtasPerSm = 2;
+// Two CTAs per SM when each fits in this much shared memory (16 consumer warps hide more
+// latency than 8); a successor launch's CTAs move in as these exit.
+constexpr int kTwoPerSmSmem = 112 * 1024;
 constexpr int kMaxSmem = 227 * 1024;
+constexpr int kMaxM = 16;
 constexpr int kBarConsumers = 1;  // named barrier of the consumer warps
-constexpr int kXBatch = 8;        // x chunks in flight per consumer thread (K <= 16384 in one batch)
+constexpr int kXBatch = 8;        // x chunks in flight per consumer thread (M = 1, K <= 16384 at once)
 
 struct TmaGemvParams {
   const __nv_bfloat16 *x;
@@ -62,27 +63,23 @@ struct TmaGemvParams {
   void *y;
   int64_t N;
   int64_t K;
-  int64_t NB;    // 16-row blocks
-  int rb_q, rb_r; // CTA c owns rb_q + (c < rb_r) row blocks starting at c * rb_q + min(c, rb_r)
-  int KT;        // 256-column k-tiles per row
-  int SPR;       // stages per row block: ceil(KT / 8)
-  int S;         // stages in the ring
-  int x_bytes;   // permuted activations: KT * 8 groups * 64 bytes
+  int64_t NB;      // 16-row blocks
+  int rb_q, rb_r;  // CTA c owns rb_q + (c < rb_r) row blocks starting at c * rb_q + min(c, rb_r)
+  int M;           // activation rows
+  int KT;          // 256-column k-tiles per row
+  int SPR;         // stages per row block: ceil(KT / 8)
+  int S;           // stages in the ring
+  int x_stride;    // bytes between activation rows in shared memory: KT * 512 + 64
+  int red_floats;  // one buffer of the row-block reduction
   int y_dtype;
-  int prefetch;  // stream codes and scales before the grid dependency resolves
-  int boxes3d;   // 1: one 3-D box per stage for the codes and one for the scales
+  int prefetch;    // stream codes and scales before the grid dependency resolves
+  int boxes3d;     // 1: one 3-D box per stage for the codes and one for the scales
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&d)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
                : "r"(addr));
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
 }
 
 // D = A * B (+ 0) and D = A * B + D for m16n8k16, bf16 inputs, fp32 accumulators.
@@ -111,17 +108,31 @@ __device__ __forceinline__ void unpack_signed(uint32_t w, uint32_t (&a)[4]) {
   a[3] = bf16x2_sub(nib_pair_bf16(w >> 12, 0x43084308u), 0x43084308u);
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__device__ __forceinline__ void store_y(const TmaGemvParams &p, int64_t m, int64_t n, float v) {
+  if (p.bias) v += __ldcg(p.bias + n);
+  if (p.y_dtype == W4_F32)
+    static_cast<float *>(p.y)[m * p.N + n] = v;
+  else
+    static_cast<__nv_bfloat16 *>(p.y)[m * p.N + n] = __float2bfloat16_rn(v);
+}
+
+// NT = 0: M = 1, x broadcast to every MMA column. NT = 1, 2: up to 8 NT activation rows,
+// one per MMA column of each n-tile.
+template <int NT>
+__global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
     gemv_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
                     const TmaGemvParams p, int32_t *err) {
+  constexpr int kTok = NT == 0 ? 1 : 8 * NT;  // token slots of the reduction buffer
+  constexpr int kAcc = NT == 0 ? 1 : NT;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte swizzle atoms
   uint8_t *xs = smem + p.S * kStageBytes;
-  float *red = reinterpret_cast<float *>(xs + p.x_bytes);
-  uint64_t *full = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(red) + kRedBytes);
+  float *red = reinterpret_cast<float *>(xs + p.M * p.x_stride);
+  uint64_t *full = reinterpret_cast<uint64_t *>(red + 2 * p.red_floats);
   uint64_t *empty = full + kMaxStages;
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kMaxStages);
+  uint64_t *x_full = empty + kMaxStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(x_full + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = static_cast<int>(blockIdx.x);
@@ -133,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kWarps);
     }
+    mbar_init(x_full, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -142,11 +154,22 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == kWarps) {
     // ---- producer: one thread issues every TMA box of the CTA's row blocks ----
     if (lane == 0) {
-      if (!p.prefetch) grid_dependency_wait();
       int slot = 0, kc = 0;
       uint32_t phase = 0;
       int32_t row = static_cast<int32_t>(rb_begin * kRowsPerBlock);
-      for (int i = 0; i < total; ++i) {
+      // weights first when they may be prefetched (they do not depend on the previous kernel)
+      const int early = p.prefetch ? (total < p.S ? total : p.S) : 0;
+      for (int i = 0; i <= total; ++i) {
+        if (NT != 0 && i == early) {
+          // x is written by the previous kernel: copy it only once that kernel has finished.
+          // (M = 1: the consumers load it themselves, in one round trip.)
+          grid_dependency_wait();
+          mbar_arrive_expect_tx(x_full, static_cast<uint32_t>(p.M * p.K * 2));
+          for (int m = 0; m < p.M; ++m)
+            bulk_copy_g2s(xs + m * p.x_stride, p.x + m * p.K, static_cast<uint32_t>(p.K * 2), x_full);
+        }
+        if (i == total) break;
+        if (NT == 0 && i == early && !p.prefetch) grid_dependency_wait();
         if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, err)) break;
         const int kt0 = kc * kKtilesPerStage;
         const int nkt = (p.KT - kt0) < kKtilesPerStage ? (p.KT - kt0) : kKtilesPerStage;
@@ -178,32 +201,51 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
 
-  // ---- consumers: x -> shared memory in B-fragment order, once per CTA ----
-  grid_dependency_wait();
-  {
-    // all loads of a thread are issued before any is used: one memory round trip, not one
-    // per chunk. Chunk c = (group, t) holds columns (8t + e, 8t + e + 4) for e = 0..3.
-    const int G = static_cast<int>(p.K / 32);
-    const int chunks = p.KT * 32;
+  // ---- consumers: x -> B-fragment order; the tail past K (up to a whole k-tile) is
+  // cleared. Chunk c of a row holds columns (8c + e, 8c + e + 4) for e = 0..3. ----
+  if (NT == 0) {
+    // one activation row: every thread issues all its loads before using any (one memory
+    // round trip), straight from global memory once the previous kernel has finished
+    grid_dependency_wait();
+    const int per_row = p.KT * 32, valid = static_cast<int>(p.K / 8);
     const uint4 *x4 = reinterpret_cast<const uint4 *>(p.x);
-    for (int base = static_cast<int>(threadIdx.x); base < chunks; base += kXBatch * 32 * kWarps) {
+    uint4 *xr = reinterpret_cast<uint4 *>(xs);
+    for (int base = static_cast<int>(threadIdx.x); base < per_row; base += kXBatch * 32 * kWarps) {
       uint4 r4[kXBatch];
 #pragma unroll
       for (int k = 0; k < kXBatch; ++k) {
         const int c = base + k * 32 * kWarps;
-        r4[k] = (c < chunks && (c >> 2) < G) ? __ldcg(x4 + c) : make_uint4(0u, 0u, 0u, 0u);
+        r4[k] = (c < valid) ? __ldcg(x4 + c) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int k = 0; k < kXBatch; ++k) {
         const int c = base + k * 32 * kWarps;
-        if (c < chunks) {
+        if (c < per_row) {
           uint4 v;
           v.x = prmt(r4[k].x, r4[k].z, 0x5410);
           v.y = prmt(r4[k].x, r4[k].z, 0x7632);
           v.z = prmt(r4[k].y, r4[k].w, 0x5410);
           v.w = prmt(r4[k].y, r4[k].w, 0x7632);
-          reinterpret_cast<uint4 *>(xs)[c] = v;
+          xr[c] = v;
         }
+      }
+    }
+  } else {
+    // several rows: one bulk copy per row (issued by the producer), permuted in place
+    mbar_wait(x_full, 0, abort_flag, err);
+    const int per_row = p.KT * 32, valid = static_cast<int>(p.K / 8);
+    for (int m = 0; m < p.M; ++m) {
+      uint4 *xr = reinterpret_cast<uint4 *>(xs + m * p.x_stride);
+      for (int c = threadIdx.x; c < per_row; c += 32 * kWarps) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (c < valid) {
+          const uint4 r4 = xr[c];
+          v.x = prmt(r4.x, r4.z, 0x5410);
+          v.y = prmt(r4.x, r4.z, 0x7632);
+          v.z = prmt(r4.y, r4.w, 0x5410);
+          v.w = prmt(r4.y, r4.w, 0x7632);
+        }
+        xr[c] = v;
       }
     }
   }
@@ -225,7 +267,19 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
   for (int q = 0; q < 4; ++q) ld_off[q] = ld_row + ((((2u * q) + ld_hi) ^ ld_xor) << 4);
 
-  float acc0 = 0.0f, acc1 = 0.0f;  // rows g and g + 8 of the current row block
+  // this lane's activation rows (one per n-tile; NT = 0: row 0 for every lane)
+  const uint4 *xrow[kAcc];
+  bool xok[kAcc];
+#pragma unroll
+  for (int j = 0; j < kAcc; ++j) {
+    const int m = NT == 0 ? 0 : 8 * j + g;
+    xok[j] = m < p.M;
+    xrow[j] = reinterpret_cast<const uint4 *>(xs + (xok[j] ? m : 0) * p.x_stride) + t;
+  }
+
+  float acc[kAcc][4];
+#pragma unroll
+  for (int j = 0; j < kAcc; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
   int buf = 0, slot = 0, kc = 0, rbl = 0;
   uint32_t phase = 0;
   int64_t row0 = rb_begin * kRowsPerBlock;
@@ -249,18 +303,24 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float s1[8] = {__uint_as_float(sh0.x), __uint_as_float(sh0.y), __uint_as_float(sh0.z),
                            __uint_as_float(sh0.w), __uint_as_float(sh1.x), __uint_as_float(sh1.y),
                            __uint_as_float(sh1.z), __uint_as_float(sh1.w)};
-      const uint4 *xk = reinterpret_cast<const uint4 *>(xs) + kt * 32 + t;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint4 xf = xk[4 * j];
+      for (int jj = 0; jj < 8; ++jj) {
         uint32_t a[4], b[4];
-        unpack_signed(w[j >> 1][(j & 1) * 2], a);      // row g
-        unpack_signed(w[j >> 1][(j & 1) * 2 + 1], b);  // row g + 8
-        float d[4];
-        mma_first(d, a[0], b[0], a[1], b[1], xf.x, xf.y);
-        mma_next(d, a[2], b[2], a[3], b[3], xf.z, xf.w);
-        acc0 = fmaf(d[0], s0[j], acc0);
-        acc1 = fmaf(d[2], s1[j], acc1);
+        unpack_signed(w[jj >> 1][(jj & 1) * 2], a);      // row g
+        unpack_signed(w[jj >> 1][(jj & 1) * 2 + 1], b);  // row g + 8
+#pragma unroll
+        for (int j = 0; j < kAcc; ++j) {
+          const uint4 xf = (NT == 0 || xok[j]) ? xrow[j][kt * 32 + 4 * jj] : make_uint4(0u, 0u, 0u, 0u);
+          float d[4];
+          mma_first(d, a[0], b[0], a[1], b[1], xf.x, xf.y);
+          mma_next(d, a[2], b[2], a[3], b[3], xf.z, xf.w);
+          acc[j][0] = fmaf(d[0], s0[jj], acc[j][0]);
+          acc[j][2] = fmaf(d[2], s1[jj], acc[j][2]);
+          if (NT != 0) {
+            acc[j][1] = fmaf(d[1], s0[jj], acc[j][1]);
+            acc[j][3] = fmaf(d[3], s1[jj], acc[j][3]);
+          }
+        }
       }
     }
     __syncwarp();
@@ -271,29 +331,40 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 
     if (++kc == p.SPR) {
-      // row block complete: the eight warps' sums meet in shared memory (fixed order)
+      // row block complete: the eight warps' sums meet in shared memory (fixed order).
+      // Layout: [warp][token][16 rows].
       kc = 0;
-      float *r = red + buf * (kWarps * kRowsPerBlock);
-      if (t == 0) {
-        r[warp * kRowsPerBlock + g] = acc0;
-        r[warp * kRowsPerBlock + g + 8] = acc1;
-      }
-      named_barrier_sync(kBarConsumers, 32 * kWarps);
-      if (warp == (rbl & (kWarps - 1)) && lane < kRowsPerBlock) {
-        const int64_t n = row0 + lane;
-        if (n < p.N) {
-          float v = 0.0f;
+      float *r = red + buf * p.red_floats;
+      if (NT == 0) {
+        if (t == 0) {
+          r[warp * kRowsPerBlock + g] = acc[0][0];
+          r[warp * kRowsPerBlock + g + 8] = acc[0][2];
+        }
+      } else {
 #pragma unroll
-          for (int w2 = 0; w2 < kWarps; ++w2) v += r[w2 * kRowsPerBlock + lane];
-          if (p.bias) v += __ldcg(p.bias + n);
-          if (p.y_dtype == W4_F32)
-            static_cast<float *>(p.y)[n] = v;
-          else
-            static_cast<__nv_bfloat16 *>(p.y)[n] = __float2bfloat16_rn(v);
+        for (int j = 0; j < kAcc; ++j) {
+          float *rw = r + (warp * kTok + 8 * j + 2 * t) * kRowsPerBlock;
+          rw[g] = acc[j][0];
+          rw[kRowsPerBlock + g] = acc[j][1];
+          rw[g + 8] = acc[j][2];
+          rw[kRowsPerBlock + g + 8] = acc[j][3];
         }
       }
-      acc0 = 0.0f;
-      acc1 = 0.0f;
+      named_barrier_sync(kBarConsumers, 32 * kWarps);
+      if (warp == (rbl & (kWarps - 1))) {
+        for (int e = lane; e < p.M * kRowsPerBlock; e += 32) {
+          const int m = e / kRowsPerBlock, rr = e % kRowsPerBlock;
+          const int64_t n = row0 + rr;
+          if (n < p.N) {
+            float v = 0.0f;
+#pragma unroll
+            for (int w2 = 0; w2 < kWarps; ++w2) v += r[(w2 * kTok + m) * kRowsPerBlock + rr];
+            store_y(p, m, n, v);
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kAcc; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
       buf ^= 1;  // the next block writes the other buffer; two barriers apart from this read
       row0 += kRowsPerBlock;
       ++rbl;
@@ -313,18 +384,25 @@ int sm_count_current() {
   return counts[dev];
 }
 
-bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem) {
-  if (lp.M != 1 || lp.asym) return false;
+// Shapes, alignment and the shared-memory plan; *ctas_per_sm is 1 or 2.
+bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_per_sm) {
+  if (lp.M < 1 || lp.M > kMaxM || lp.asym) return false;
   if (lp.K % 128 != 0 || lp.N > 0x7fffffffLL) return false;  // TMA: 16-byte row strides, int32 rows
   if (lp.y_dtype != W4_BF16 && lp.y_dtype != W4_F32) return false;
   const uintptr_t a = reinterpret_cast<uintptr_t>(lp.codes) | reinterpret_cast<uintptr_t>(lp.scales) |
                       reinterpret_cast<uintptr_t>(lp.x);
   if (a % 16 != 0) return false;
   const int64_t KT = (lp.K + 255) / 256;
-  const int64_t x_bytes = KT * 512;
-  const int64_t fixed = kAlignSlack + x_bytes + kRedBytes + kBarBytes;
-  int64_t S = (kCoResidentSmem - fixed) / kStageBytes;
-  if (S < 4) S = (kMaxSmem - fixed) / kStageBytes;  // long rows: give up co-residency for depth
+  const int64_t x_stride = KT * 512 + 64;  // the 64 bytes keep two rows of a lane quad on distinct banks
+  const int64_t tok = lp.M == 1 ? 1 : (lp.M <= 8 ? 8 : 16);
+  const int64_t red_floats = kWarps * tok * kRowsPerBlock;
+  const int64_t fixed = kAlignSlack + lp.M * x_stride + 2 * red_floats * 4 + kBarBytes;
+  int64_t S = (kTwoPerSmSmem - fixed) / kStageBytes;
+  int per_sm = 2;
+  if (S < 4) {  // long rows or many activation rows: one CTA per SM, a deeper ring
+    S = (kMaxSmem - fixed) / kStageBytes;
+    per_sm = 1;
+  }
   if (S > kMaxStages) S = kMaxStages;
   if (S < 2) return false;
   q->x = lp.x;
@@ -334,16 +412,21 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem) {
   q->K = lp.K;
   q->NB = (lp.N + kRowsPerBlock - 1) / kRowsPerBlock;
   if (q->NB >= (int64_t(1) << 31) / 64) return false;
+  q->M = static_cast<int>(lp.M);
   q->KT = static_cast<int>(KT);
   q->SPR = static_cast<int>((KT + kKtilesPerStage - 1) / kKtilesPerStage);
   q->S = static_cast<int>(S);
-  q->x_bytes = static_cast<int>(x_bytes);
+  q->x_stride = static_cast<int>(x_stride);
+  q->red_floats = static_cast<int>(red_floats);
   q->y_dtype = lp.y_dtype;
   q->prefetch = 0;
+  q->boxes3d = 0;
   *smem = static_cast<int>(fixed + S * kStageBytes);
+  *ctas_per_sm = per_sm;
   return true;
 }
 
+template <int NT>
 cudaError_t ensure_smem_attr() {
   static std::mutex mu;
   static bool done[64] = {};
@@ -353,25 +436,43 @@ cudaError_t ensure_smem_attr() {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (!done[dev]) {
-    e = cudaFuncSetAttribute(gemv_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    e = cudaFuncSetAttribute(gemv_tma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return e;
     done[dev] = true;
   }
   return cudaSuccess;
 }
 
+template <int NT>
+cudaError_t launch_typed(const CUtensorMap &mc, const CUtensorMap &ms, const TmaGemvParams &q, int smem, int grid,
+                         int32_t *err, cudaStream_t stream) {
+  cudaError_t e = ensure_smem_attr<NT>();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_tma_kernel<NT>, mc, ms, q, err);
+}
+
 }  // namespace
 
 bool gemv_tma_supports(const LinearParams &p) {
   TmaGemvParams q;
-  int smem;
-  return make_params(p, &q, &smem) && encode_fn() != nullptr;
+  int smem, per_sm;
+  return make_params(p, &q, &smem, &per_sm) && encode_fn() != nullptr;
 }
 
 cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, int32_t *err, cudaStream_t stream) {
   TmaGemvParams q;
-  int smem = 0;
-  if (!make_params(lp, &q, &smem)) return cudaErrorNotSupported;
+  int smem = 0, per_sm = 1;
+  if (!make_params(lp, &q, &smem, &per_sm)) return cudaErrorNotSupported;
   q.prefetch = prefetch ? 1 : 0;
   const int64_t P = lp.K / 2, G = lp.K / 32;
   CUtensorMap mc, ms;
@@ -389,23 +490,13 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, int32_t *err,
        !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, G, lp.N, G * 4, 32, kRowsPerBlock,
                     CU_TENSOR_MAP_SWIZZLE_128B)))
     return cudaErrorInvalidValue;
-  cudaError_t e = ensure_smem_attr();
-  if (e != cudaSuccess) return e;
-  const int64_t slots = static_cast<int64_t>(sm_count_current()) * kCtasPerSm;
+  const int64_t slots = static_cast<int64_t>(sm_count_current()) * per_sm;
   const int64_t grid = q.NB < slots ? q.NB : slots;
   q.rb_q = static_cast<int>(q.NB / grid);
   q.rb_r = static_cast<int>(q.NB % grid);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_tma_kernel, mc, ms, q, err);
+  if (lp.M == 1) return launch_typed<0>(mc, ms, q, smem, static_cast<int>(grid), err, stream);
+  if (lp.M <= 8) return launch_typed<1>(mc, ms, q, smem, static_cast<int>(grid), err, stream);
+  return launch_typed<2>(mc, ms, q, smem, static_cast<int>(grid), err, stream);
 }
 
 }  // namespace w4i

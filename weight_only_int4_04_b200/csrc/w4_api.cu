@@ -56,11 +56,11 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
   int32_t *err = nullptr;
   const w4_status st = symbol_ptr(&err, g_device_error);
   if (st != W4_OK) return st;
-  // M dispatch: M = 1 -> the TMA-fed tensor-core GEMV (symmetric codes, K a multiple of
-  // 128), else the register-streaming GEMV; M <= 16 -> the tensor-core decode kernel
-  // (bulk-copy slot ring, mma.sync); larger M -> the tcgen05 GEMM; the other GEMV kernels and
-  // the generic kernel take the shapes the fast paths cannot (unaligned rows, odd widths,
-  // unsorted act-order maps). W4_GEMV=rows|stream|mma picks an alternative M = 1 kernel (for
+  // M dispatch: M <= 16 -> the TMA-fed tensor-core GEMV (symmetric codes, K a multiple of
+  // 128, activations that fit in shared memory), else for M = 1 the register-streaming GEMV
+  // and for M <= 16 the bulk-copy mma.sync kernel; larger M -> the tcgen05 GEMM; the other
+  // kernels take the shapes the fast paths cannot (unaligned rows, odd widths, unsorted
+  // act-order maps). W4_GEMV=rows|stream|mma picks an alternative small-M kernel (for
   // comparisons only).
   static const int m1_kernel = [] {
     const char *v = getenv("W4_GEMV");

@@ -56,10 +56,11 @@ bool gemv_rows_supports(const LinearParams &p);
 // bulk-copy slot ring; the main decode path.
 cudaError_t launch_gemv_mma(const LinearParams &p, int32_t *err, cudaStream_t stream);
 bool gemv_mma_supports(const LinearParams &p);
-// Decode GEMV (M = 1, symmetric codes, K a multiple of 128, 16-byte aligned arrays) on
-// register-fed tensor cores with a TMA stage ring; launched with programmatic stream
-// serialization. `prefetch` lets it stream codes and scales before the previous kernel of
-// the stream has finished (x and y are touched only after it has).
+// Decode GEMV / small-M linear (M <= 16, symmetric codes, K a multiple of 128, 16-byte
+// aligned arrays, activations that fit in shared memory) on register-fed tensor cores with
+// a TMA stage ring; launched with programmatic stream serialization. `prefetch` lets it
+// stream codes and scales before the previous kernel of the stream has finished (x and y
+// are touched only after it has).
 cudaError_t launch_gemv_tma(const LinearParams &p, bool prefetch, int32_t *err, cudaStream_t stream);
 bool gemv_tma_supports(const LinearParams &p);
 // Tensor-core GEMM (tcgen05, TMA, TMEM) for larger M, aligned rows. The asymmetric
