@@ -21,6 +21,8 @@
 // MMA. All waits are bounded (see w4_sync.cuh).
 #include <cuda.h>
 
+#include <mutex>
+
 #include "w4_tc.cuh"
 #include "w4_tmap.h"
 
@@ -29,34 +31,34 @@ namespace w4i {
 namespace {
 
 constexpr int BM_W = 128;  // weight rows per tile (MMA M)
-constexpr int BN_X = 256;  // activation rows per tile (MMA N)
 constexpr int BK = 64;     // K per stage: one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
 constexpr int kThreads = 320;
 constexpr int kDequantWarp0 = 2;
 
 constexpr int A_BYTES = BM_W * BK * 2;    // 16 KB
-constexpr int B_BYTES = BN_X * BK * 2;    // 32 KB
 constexpr int C_BYTES = BM_W * (BK / 2);  // 4 KB of codes
 constexpr int S_BYTES = BM_W * 4 * 4;     // 2 KB: 4 scale columns per row
 constexpr int Z_BYTES = BM_W * 16;        // 2 KB: 16 zero-point columns per row (asymmetric)
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_S = OFF_C + STAGES * C_BYTES;
-constexpr int OFF_Z = OFF_S + STAGES * S_BYTES;
-template <bool ASYM>
-__host__ __device__ constexpr int off_gstage() { return ASYM ? OFF_Z + STAGES * Z_BYTES : OFF_Z; }
-constexpr int kMaxStagesAsym = 512;        // K <= 32768 on the asymmetric path
-template <bool ASYM>
-__host__ __device__ constexpr int off_bar() { return off_gstage<ASYM>() + (ASYM ? 2 * kMaxStagesAsym : 0); }
-template <bool ASYM>
-__host__ __device__ constexpr int smem_bytes() { return off_bar<ASYM>() + 256 + 1024; }  // barriers + 1 KB alignment slack
-static_assert(smem_bytes<true>() <= 227 * 1024, "asymmetric GEMM exceeds the shared-memory budget");
-static_assert(smem_bytes<false>() <= 227 * 1024, "GEMM exceeds the shared-memory budget");
-template <bool ASYM>
-__host__ __device__ constexpr uint32_t tx_bytes() { return B_BYTES + C_BYTES + S_BYTES + (ASYM ? Z_BYTES : 0); }
-constexpr uint32_t TMEM_COLS = BN_X;
+constexpr int kMaxStagesAsym = 512;       // K <= 32768 on the asymmetric path
+
+// Shared-memory plan for BN activation rows per tile (MMA N = BN: 64 for the mid-M range,
+// 256 for prefill); a narrower tile leaves room for a deeper ring.
+template <bool ASYM, int BN>
+struct TcLayout {
+  static constexpr int STAGES = BN <= 64 ? 6 : 4;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_S = OFF_C + STAGES * C_BYTES;
+  static constexpr int OFF_Z = OFF_S + STAGES * S_BYTES;
+  static constexpr int OFF_G = ASYM ? OFF_Z + STAGES * Z_BYTES : OFF_Z;
+  static constexpr int OFF_BAR = OFF_G + (ASYM ? 2 * kMaxStagesAsym : 0);
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + 1 KB alignment slack
+  static constexpr uint32_t TX = B_BYTES + C_BYTES + S_BYTES + (ASYM ? Z_BYTES : 0);
+  static constexpr uint32_t TMEM_COLS = BN;
+  static_assert(SMEM <= 227 * 1024, "GEMM exceeds the shared-memory budget");
+};
 
 struct TcParams {
   const float *bias;
@@ -72,17 +74,19 @@ struct TcParams {
   int n_groups;
 };
 
-template <bool ASYM>
+template <bool ASYM, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
                    const __grid_constant__ CUtensorMap tmap_scales, const __grid_constant__ CUtensorMap tmap_zeros,
                    const TcParams p, int32_t *err) {
+  using L = TcLayout<ASYM, BN>;
+  constexpr int STAGES = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base (the 128-byte swizzle atoms must start on 1024-byte boundaries)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint64_t *full_load = reinterpret_cast<uint64_t *>(smem + off_bar<ASYM>());
-  int16_t *gstage = reinterpret_cast<int16_t *>(smem + off_gstage<ASYM>());
+  uint64_t *full_load = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
+  int16_t *gstage = reinterpret_cast<int16_t *>(smem + L::OFF_G);
   uint64_t *full_a = full_load + STAGES;
   uint64_t *empty = full_a + STAGES;
   uint64_t *acc_full = empty + STAGES;
@@ -91,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BM_W;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * BN_X;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * BN;
   const int KB = static_cast<int>((p.K + BK - 1) / BK);
 
   if (threadIdx.x == 0) {
@@ -113,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       gstage[kb] = static_cast<int16_t>(g0 == __ldg(p.g_idx + __ldg(p.perm + last)) ? g0 : -1);
     }
   }
-  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (warp == 1) tmem_alloc(tmem_slot, L::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -125,25 +129,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = kb % STAGES;
         const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err)) break;
-        mbar_arrive_expect_tx(&full_load[s], tx_bytes<ASYM>());
-        tma_load_2d(smem + OFF_B + s * B_BYTES, &tmap_x, kb * BK, static_cast<int32_t>(m0), &full_load[s]);
-        tma_load_2d(smem + OFF_C + s * C_BYTES, &tmap_codes, kb * (BK / 2), static_cast<int32_t>(n0),
+        mbar_arrive_expect_tx(&full_load[s], L::TX);
+        tma_load_2d(smem + L::OFF_B + s * L::B_BYTES, &tmap_x, kb * BK, static_cast<int32_t>(m0), &full_load[s]);
+        tma_load_2d(smem + L::OFF_C + s * C_BYTES, &tmap_codes, kb * (BK / 2), static_cast<int32_t>(n0),
                     &full_load[s]);
         if (!ASYM) {
-          tma_load_2d(smem + OFF_S + s * S_BYTES, &tmap_scales, 4 * (kb / 2), static_cast<int32_t>(n0),
+          tma_load_2d(smem + L::OFF_S + s * S_BYTES, &tmap_scales, 4 * (kb / 2), static_cast<int32_t>(n0),
                       &full_load[s]);
         } else {
           const int gs = gstage[kb] < 0 ? 0 : gstage[kb];
-          tma_load_2d(smem + OFF_S + s * S_BYTES, &tmap_scales, gs & ~3, static_cast<int32_t>(n0), &full_load[s]);
-          tma_load_2d(smem + OFF_Z + s * Z_BYTES, &tmap_zeros, gs & ~15, static_cast<int32_t>(n0), &full_load[s]);
+          tma_load_2d(smem + L::OFF_S + s * S_BYTES, &tmap_scales, gs & ~3, static_cast<int32_t>(n0), &full_load[s]);
+          tma_load_2d(smem + L::OFF_Z + s * Z_BYTES, &tmap_zeros, gs & ~15, static_cast<int32_t>(n0), &full_load[s]);
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM_W, BN_X);
-      const uint32_t a_base = smem_u32(smem + OFF_A);
-      const uint32_t b_base = smem_u32(smem + OFF_B);
+      constexpr uint32_t idesc = umma_idesc_bf16_f32(BM_W, BN);
+      const uint32_t a_base = smem_u32(smem + L::OFF_A);
+      const uint32_t b_base = smem_u32(smem + L::OFF_B);
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t ad = umma_desc_sw128(a_base + s * A_BYTES + kk * 32);
-          const uint64_t bd = umma_desc_sw128(b_base + s * B_BYTES + kk * 32);
+          const uint64_t bd = umma_desc_sw128(b_base + s * L::B_BYTES + kk * 32);
           umma_bf16(tmem_d, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&empty[s]);
@@ -165,25 +169,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                      // TMEM lane quarter this warp may access
     const int half = (warp - kDequantWarp0) >> 2;  // which 32 of the stage's 64 columns
     const int r = 32 * q + lane;                 // weight row inside the tile
-    const uint32_t a_row = smem_u32(smem + OFF_A) + r * 128;
+    const uint32_t a_row = smem_u32(smem + L::OFF_A) + r * 128;
     for (int kb = 0; kb < KB; ++kb) {
       const int s = kb % STAGES;
       const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
       mbar_wait(&full_load[s], ph, abort_flag, err);
-      const uint4 cw = *reinterpret_cast<const uint4 *>(smem + OFF_C + s * C_BYTES + r * 32 + 16 * half);
+      const uint4 cw = *reinterpret_cast<const uint4 *>(smem + L::OFF_C + s * C_BYTES + r * 32 + 16 * half);
       const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
       float sc;
       uint32_t xorc = 0x08080808u;
       uint64_t nb2 = neg_bias_pair(8u);
       int gs = 0;
       if (!ASYM) {
-        sc = reinterpret_cast<const float *>(smem + OFF_S + s * S_BYTES)[r * 4 + (kb & 1) * 2 + half];
+        sc = reinterpret_cast<const float *>(smem + L::OFF_S + s * S_BYTES)[r * 4 + (kb & 1) * 2 + half];
       } else {
         gs = gstage[kb];
         const int gsc = gs < 0 ? 0 : gs;
-        sc = reinterpret_cast<const float *>(smem + OFF_S + s * S_BYTES)[r * 4 + (gsc & 3)];
+        sc = reinterpret_cast<const float *>(smem + L::OFF_S + s * S_BYTES)[r * 4 + (gsc & 3)];
         const uint32_t z = static_cast<uint32_t>(
-            reinterpret_cast<const uint8_t *>(smem + OFF_Z + s * Z_BYTES)[r * 16 + (gsc & 15)]) & 15u;
+            reinterpret_cast<const uint8_t *>(smem + L::OFF_Z + s * Z_BYTES)[r * 16 + (gsc & 15)]) & 15u;
         xorc = 0u;
         nb2 = neg_bias_pair(z);
       }
@@ -232,8 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t n = n0 + r;
     const float b = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      const int col0 = 128 * half + 32 * c;
+    for (int c = 0; c < BN / 64; ++c) {
+      const int col0 = (BN / 2) * half + 32 * c;
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(32 * q) << 16) + col0, v);
       if (n < p.N) {
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_d, TMEM_COLS);
+    tmem_dealloc(tmem_d, L::TMEM_COLS);
   }
 }
 
@@ -274,7 +278,7 @@ bool gemm_tc_supports(const LinearParams &p) {
                       (p.asym ? reinterpret_cast<uintptr_t>(p.zeros) : 0) |
                       (p.asym ? 0 : reinterpret_cast<uintptr_t>(p.x));
   if (a % 16 != 0) return false;
-  if ((p.M + BN_X - 1) / BN_X > 65535 || (p.N + BM_W - 1) / BM_W > 0x7fffffffLL) return false;
+  if ((p.M + 255) / 256 > 65535 || (p.N + BM_W - 1) / BM_W > 0x7fffffffLL) return false;
   return encode_fn() != nullptr;
 }
 
@@ -302,6 +306,28 @@ size_t gemm_tc_asym_workspace(int64_t M, int64_t K) {
   return static_cast<size_t>(((M * K * 2 + 255) / 256) * 256);
 }
 
+template <bool ASYM, int BN>
+cudaError_t launch_typed(dim3 grid, const CUtensorMap &mx, const CUtensorMap &mc, const CUtensorMap &ms,
+                         const CUtensorMap &mz, const TcParams &tp, int32_t *err, cudaStream_t stream) {
+  using L = TcLayout<ASYM, BN>;
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+      e = cudaFuncSetAttribute(gemm_tc_kernel<ASYM, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM);
+      if (e != cudaSuccess) return e;
+      done[dev] = true;
+    }
+  }
+  gemm_tc_kernel<ASYM, BN><<<grid, kThreads, L::SMEM, stream>>>(mx, mc, ms, mz, tp, err);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t stream, void *workspace) {
   if (!gemm_tc_supports(p)) return cudaErrorNotSupported;
   const int64_t P = (p.K + 1) / 2, G = (p.K + 31) / 32;
@@ -316,8 +342,11 @@ cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t str
     xsrc = xg;
   }
   const int64_t SG = p.asym ? p.n_groups : G;
+  // MMA N = activation rows per tile: 64 up to M = 64 (the mid-M range, where the weight
+  // stream dominates and a wider tile would only multiply idle tensor work), else 256
+  const int bn = p.M <= 64 ? 64 : 256;
   CUtensorMap mx, mc, ms, mz;
-  if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xsrc, p.K, p.M, p.K * 2, BK, BN_X,
+  if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xsrc, p.K, p.M, p.K * 2, BK, bn,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.codes, P, p.N, P, BK / 2, BM_W, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.scales, SG, p.N, SG * 4, 4, BM_W,
@@ -330,27 +359,13 @@ cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t str
     mz = ms;  // unused by the symmetric kernel
   }
   TcParams tp{p.bias, p.y, p.M, p.N, p.K, p.y_dtype, p.g_idx, p.perm, p.scales, p.zeros, p.n_groups};
-  const dim3 grid(static_cast<unsigned>((p.N + BM_W - 1) / BM_W), static_cast<unsigned>((p.M + BN_X - 1) / BN_X));
+  const dim3 grid(static_cast<unsigned>((p.N + BM_W - 1) / BM_W), static_cast<unsigned>((p.M + bn - 1) / bn));
   if (p.asym) {
-    static bool attr = false;
-    if (!attr) {
-      const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem_bytes<true>());
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    gemm_tc_kernel<true><<<grid, kThreads, smem_bytes<true>(), stream>>>(mx, mc, ms, mz, tp, err);
-  } else {
-    static bool attr = false;
-    if (!attr) {
-      const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 smem_bytes<false>());
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
-    gemm_tc_kernel<false><<<grid, kThreads, smem_bytes<false>(), stream>>>(mx, mc, ms, mz, tp, err);
+    if (bn == 64) return launch_typed<true, 64>(grid, mx, mc, ms, mz, tp, err, stream);
+    return launch_typed<true, 256>(grid, mx, mc, ms, mz, tp, err, stream);
   }
-  return cudaGetLastError();
+  if (bn == 64) return launch_typed<false, 64>(grid, mx, mc, ms, mz, tp, err, stream);
+  return launch_typed<false, 256>(grid, mx, mc, ms, mz, tp, err, stream);
 }
 
 }  // namespace w4i
