@@ -123,9 +123,10 @@ w4_status w4_linear(const void *x, int64_t M, const uint8_t *codes, const float 
 size_t w4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /* Workspace bytes w4_linear_asym_gidx uses for this shape when its codes are prepared
- * (perm given): for M above the decode sizes the activations are gathered through perm into
- * the workspace (M * K bf16, rounded up to 256 bytes) and a tensor-core GEMM runs. A call
- * given less (or no) workspace still succeeds on a slower kernel. */
+ * (perm given): the activations are gathered through perm into the workspace once per call
+ * (M * K bf16, rounded up to 256 bytes) for the tensor-core GEMM (larger M) and for the decode
+ * kernel (K a multiple of 128). A call given less (or no) workspace still succeeds on a
+ * slower kernel. */
 size_t w4_linear_asym_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t n_groups);
 
 /*

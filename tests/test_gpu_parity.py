@@ -390,6 +390,21 @@ def test_asym_small(w4, prepared, M, NKG):
     _asym_check(w4, c, prepared)
 
 
+@pytest.mark.parametrize("M", [1, 3, 9, 16])
+@pytest.mark.parametrize("NK", [(48, 512), (40, 1280)])
+def test_asym_ragged_groups(w4, M, NK):
+    """Act-order groups of uneven sizes (g_idx drawn at random, not a permutation of equal
+    groups): after sorting, group boundaries fall inside 32-column chunks, which the
+    tensor-core path handles column by column."""
+    N, K = NK
+    c = workloads.asym_case(M=M, N=N, K=K, group=128, seed=900 + M + K)
+    n_groups = 7
+    c["g_idx"] = np.random.default_rng(M + K).integers(0, n_groups, size=K).astype(np.int32)
+    c["n_groups"] = n_groups
+    _asym_check(w4, c, prepared=True)
+    _asym_check(w4, c, prepared=False)
+
+
 @pytest.mark.parametrize("M", workloads.ASYM_M)
 def test_asym_full_size(w4, M):
     c = workloads.asym_case(M=M)

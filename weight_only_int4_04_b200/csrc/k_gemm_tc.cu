@@ -302,6 +302,14 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const __nv_bfloat16 *__re
   }
 }
 
+cudaError_t launch_gather_x(const __nv_bfloat16 *x, const int32_t *perm, int64_t M, int64_t K, __nv_bfloat16 *xg,
+                            cudaStream_t stream) {
+  int64_t blocks = (M * (K / 8) + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  gather_x_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, perm, M, K, xg);
+  return cudaGetLastError();
+}
+
 size_t gemm_tc_asym_workspace(int64_t M, int64_t K) {
   return static_cast<size_t>(((M * K * 2 + 255) / 256) * 256);
 }
@@ -336,9 +344,8 @@ cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t str
     // act-order: the activations are gathered once into the workspace in sorted column order
     if (workspace == nullptr || reinterpret_cast<uintptr_t>(workspace) % 16 != 0) return cudaErrorInvalidValue;
     __nv_bfloat16 *xg = static_cast<__nv_bfloat16 *>(workspace);
-    int64_t blocks = (p.M * (p.K / 8) + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
-    gather_x_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.x, p.perm, p.M, p.K, xg);
+    const cudaError_t e = launch_gather_x(p.x, p.perm, p.M, p.K, xg, stream);
+    if (e != cudaSuccess) return e;
     xsrc = xg;
   }
   const int64_t SG = p.asym ? p.n_groups : G;

@@ -61,6 +61,14 @@ struct TmaGemvParams {
   const __nv_bfloat16 *x;
   const float *bias;
   void *y;
+  // asymmetric act-order only (codes sorted by group, x gathered through perm)
+  const float *scales;    // [N, n_groups]
+  const int8_t *zeros;    // [N, n_groups]
+  const int32_t *g_idx;   // [K], group of an original column
+  const int32_t *perm;    // [K], original column at each sorted position
+  int n_groups;
+  int asym_staged;        // 1: each stage also carries the row block's scales and zero points
+  int x_sorted;           // 1: x already gathered into sorted column order (by the caller)
   int64_t N;
   int64_t K;
   int64_t NB;      // 16-row blocks
@@ -116,12 +124,64 @@ __device__ __forceinline__ void store_y(const TmaGemvParams &p, int64_t m, int64
     static_cast<__nv_bfloat16 *>(p.y)[m * p.N + n] = __float2bfloat16_rn(v);
 }
 
+// One sorted 32-column chunk whose columns belong to two or more groups (asymmetric
+// act-order codes with group boundaries that are not multiples of 32): lane (g, t) takes
+// its 8 columns of rows g and g + 8 on CUDA cores, exact per-column dequantization, and
+// the four lanes of a row pool their sums. Returns the chunk's sum for (row, token)
+// through `out[r][m]` (r = 0: row g, 1: row g + 8) in every lane of the row.
+template <int MT>
+__device__ void mixed_chunk(const TmaGemvParams &p, int64_t row_g, int c, int t, uint32_t w_g, uint32_t w_g8,
+                            const uint8_t *xs, float (&out)[2][MT]) {
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) out[r][m] = 0.0f;
+  for (int e = 0; e < 8; ++e) {
+    const int64_t col = 32 * static_cast<int64_t>(c) + 8 * t + e;
+    if (col >= p.K) break;
+    const int gc = __ldg(p.g_idx + __ldg(p.perm + col));
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int64_t n = row_g + 8 * r;
+      if (n >= p.N) continue;
+      const int u = static_cast<int>(((r ? w_g8 : w_g) >> (4 * e)) & 15u);
+      const float wv = __fmul_rn(static_cast<float>(u - __ldg(p.zeros + n * p.n_groups + gc)),
+                                 __ldg(p.scales + n * p.n_groups + gc));
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        if (m >= p.M) break;
+        // x chunk (c, t) in fragment order: pairs (x0,x4) (x1,x5) (x2,x6) (x3,x7)
+        const uint32_t pair = reinterpret_cast<const uint32_t *>(xs + m * p.x_stride)[(c * 4 + t) * 4 + (e & 3)];
+        const float xv = __uint_as_float((e < 4 ? (pair & 0xFFFFu) : (pair >> 16)) << 16);
+        out[r][m] = fmaf(wv, xv, out[r][m]);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      out[r][m] += __shfl_xor_sync(0xffffffffu, out[r][m], 1);
+      out[r][m] += __shfl_xor_sync(0xffffffffu, out[r][m], 2);
+    }
+}
+
+// One code word of unsigned nibbles -> the exact integers u - z (z: the row's zero point
+// of the chunk's group, as the bf16x2 pair (128 + z, 128 + z)).
+__device__ __forceinline__ void unpack_asym(uint32_t w, uint32_t zz, uint32_t (&a)[4]) {
+  a[0] = bf16x2_sub(nib_pair_bf16(w, 0x43004300u), zz);
+  a[1] = bf16x2_sub(nib_pair_bf16(w >> 4, 0x43004300u), zz);
+  a[2] = bf16x2_sub(nib_pair_bf16(w >> 8, 0x43004300u), zz);
+  a[3] = bf16x2_sub(nib_pair_bf16(w >> 12, 0x43004300u), zz);
+}
+
 // NT = 0: M = 1, x broadcast to every MMA column. NT = 1, 2: up to 8 NT activation rows,
-// one per MMA column of each n-tile.
-template <int NT>
+// one per MMA column of each n-tile. ASYM: unsigned codes sorted by group (act-order),
+// per-(row, group) scale and zero point read through a per-CTA group table.
+template <int NT, bool ASYM>
 __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
     gemv_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
-                    const TmaGemvParams p, int32_t *err) {
+                    const __grid_constant__ CUtensorMap tm_zeros, const TmaGemvParams p, int32_t *err) {
   constexpr int kTok = NT == 0 ? 1 : 8 * NT;  // token slots of the reduction buffer
   constexpr int kAcc = NT == 0 ? 1 : NT;
   extern __shared__ uint8_t smem_raw[];
@@ -129,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
   uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte swizzle atoms
   uint8_t *xs = smem + p.S * kStageBytes;
   float *red = reinterpret_cast<float *>(xs + p.M * p.x_stride);
-  uint64_t *full = reinterpret_cast<uint64_t *>(red + 2 * p.red_floats);
+  int32_t *gtab = reinterpret_cast<int32_t *>(red + 2 * p.red_floats);  // ASYM: group of each chunk
+  uint64_t *full = reinterpret_cast<uint64_t *>(gtab + (ASYM ? p.KT * 8 : 0));
   uint64_t *empty = full + kMaxStages;
   uint64_t *x_full = empty + kMaxStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(x_full + 1);
@@ -160,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
       // weights first when they may be prefetched (they do not depend on the previous kernel)
       const int early = p.prefetch ? (total < p.S ? total : p.S) : 0;
       for (int i = 0; i <= total; ++i) {
-        if (NT != 0 && i == early) {
+        if (NT != 0 && (!ASYM || p.x_sorted) && i == early) {
           // x is written by the previous kernel: copy it only once that kernel has finished.
           // (M = 1: the consumers load it themselves, in one round trip.)
           grid_dependency_wait();
@@ -169,13 +230,29 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
             bulk_copy_g2s(xs + m * p.x_stride, p.x + m * p.K, static_cast<uint32_t>(p.K * 2), x_full);
         }
         if (i == total) break;
-        if (NT == 0 && i == early && !p.prefetch) grid_dependency_wait();
+        if ((NT == 0 || (ASYM && !p.x_sorted)) && i == early && !p.prefetch) grid_dependency_wait();
         if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, err)) break;
         const int kt0 = kc * kKtilesPerStage;
         const int nkt = (p.KT - kt0) < kKtilesPerStage ? (p.KT - kt0) : kKtilesPerStage;
         const int nsb = (nkt + 3) / 4;
         uint8_t *st = smem + slot * kStageBytes;
-        if (p.boxes3d) {
+        if (ASYM) {
+          // codes, and (staged layout) the row block's scales and zero points of every group
+          const uint32_t sz = p.asym_staged ? static_cast<uint32_t>(kRowsPerBlock * p.n_groups * 5) : 0u;
+          if (p.boxes3d) {
+            mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(kKtilesPerStage * kCodeBox) + sz);
+            tma_load_3d(st, &tm_codes, 0, row, kt0, &full[slot]);
+          } else {
+            mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox) + sz);
+            for (int j = 0; j < nkt; ++j)
+              tma_load_2d(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot]);
+          }
+          if (p.asym_staged) {
+            uint8_t *sa = st + kKtilesPerStage * kCodeBox;
+            tma_load_2d(sa, &tm_scales, 0, row, &full[slot]);
+            tma_load_2d(sa + kRowsPerBlock * p.n_groups * 4, &tm_zeros, 0, row, &full[slot]);
+          }
+        } else if (p.boxes3d) {
           // whole-stage boxes; k-tiles past the row end read as zeros (and count as bytes)
           mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(kStageBytes));
           tma_load_3d(st, &tm_codes, 0, row, kt0, &full[slot]);
@@ -203,8 +280,52 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
 
   // ---- consumers: x -> B-fragment order; the tail past K (up to a whole k-tile) is
   // cleared. Chunk c of a row holds columns (8c + e, 8c + e + 4) for e = 0..3. ----
-  if (NT == 0) {
-    // one activation row: every thread issues all its loads before using any (one memory
+  if (ASYM) {
+    // act-order: the group of every sorted 32-column chunk (-1: the chunk straddles groups;
+    // -2: past K). perm and g_idx are weights (constant).
+    for (int c = threadIdx.x; c < p.KT * 8; c += 32 * kWarps) {
+      int gv = -2;
+      if (32 * static_cast<int64_t>(c) < p.K) {
+        const int64_t c0 = 32 * static_cast<int64_t>(c);
+        const int64_t c1 = (c0 + 31 < p.K) ? c0 + 31 : p.K - 1;
+        const int g0 = __ldg(p.g_idx + __ldg(p.perm + c0));
+        gv = g0 == __ldg(p.g_idx + __ldg(p.perm + c1)) ? g0 : -1;
+      }
+      gtab[c] = gv;
+    }
+  }
+  if (ASYM && !p.x_sorted) {
+    // x gathered through perm here (without a caller-side gather: every CTA gathers all of x)
+    const int per_row = p.KT * 32, valid = static_cast<int>(p.K / 8);
+    grid_dependency_wait();
+    const uint16_t *xb = reinterpret_cast<const uint16_t *>(p.x);
+    for (int c = threadIdx.x; c < per_row; c += 32 * kWarps) {
+      int32_t col[8];
+      if (c < valid) {
+        const int4 p0 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c);
+        const int4 p1 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c + 1);
+        col[0] = p0.x, col[1] = p0.y, col[2] = p0.z, col[3] = p0.w;
+        col[4] = p1.x, col[5] = p1.y, col[6] = p1.z, col[7] = p1.w;
+      }
+      for (int m = 0; m < p.M; ++m) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (c < valid) {
+          uint32_t r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            r[i] = static_cast<uint32_t>(__ldcg(xb + m * p.K + col[2 * i])) |
+                   (static_cast<uint32_t>(__ldcg(xb + m * p.K + col[2 * i + 1])) << 16);
+          v.x = prmt(r[0], r[2], 0x5410);
+          v.y = prmt(r[0], r[2], 0x7632);
+          v.z = prmt(r[1], r[3], 0x5410);
+          v.w = prmt(r[1], r[3], 0x7632);
+        }
+        reinterpret_cast<uint4 *>(xs + m * p.x_stride)[c] = v;
+      }
+    }
+  } else if (NT == 0) {
+    // one activation row (already in sorted order for act-order codes): every thread issues
+    // all its loads before using any (one memory
     // round trip), straight from global memory once the previous kernel has finished
     grid_dependency_wait();
     const int per_row = p.KT * 32, valid = static_cast<int>(p.K / 8);
@@ -292,33 +413,110 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
       uint32_t w[4][4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) ldsm_x4(cb + ld_off[q], w[q]);
-      const uint8_t *sp = smem + slot * kStageBytes + sbox;
-      const uint4 sg0 = *reinterpret_cast<const uint4 *>(sp + s_lo);
-      const uint4 sg1 = *reinterpret_cast<const uint4 *>(sp + s_hi);
-      const uint4 sh0 = *reinterpret_cast<const uint4 *>(sp + 1024 + s_lo);
-      const uint4 sh1 = *reinterpret_cast<const uint4 *>(sp + 1024 + s_hi);
-      const float s0[8] = {__uint_as_float(sg0.x), __uint_as_float(sg0.y), __uint_as_float(sg0.z),
-                           __uint_as_float(sg0.w), __uint_as_float(sg1.x), __uint_as_float(sg1.y),
-                           __uint_as_float(sg1.z), __uint_as_float(sg1.w)};
-      const float s1[8] = {__uint_as_float(sh0.x), __uint_as_float(sh0.y), __uint_as_float(sh0.z),
-                           __uint_as_float(sh0.w), __uint_as_float(sh1.x), __uint_as_float(sh1.y),
-                           __uint_as_float(sh1.z), __uint_as_float(sh1.w)};
+      if (!ASYM) {
+        const uint8_t *sp = smem + slot * kStageBytes + sbox;
+        const uint4 sg0 = *reinterpret_cast<const uint4 *>(sp + s_lo);
+        const uint4 sg1 = *reinterpret_cast<const uint4 *>(sp + s_hi);
+        const uint4 sh0 = *reinterpret_cast<const uint4 *>(sp + 1024 + s_lo);
+        const uint4 sh1 = *reinterpret_cast<const uint4 *>(sp + 1024 + s_hi);
+        const float s0[8] = {__uint_as_float(sg0.x), __uint_as_float(sg0.y), __uint_as_float(sg0.z),
+                             __uint_as_float(sg0.w), __uint_as_float(sg1.x), __uint_as_float(sg1.y),
+                             __uint_as_float(sg1.z), __uint_as_float(sg1.w)};
+        const float s1[8] = {__uint_as_float(sh0.x), __uint_as_float(sh0.y), __uint_as_float(sh0.z),
+                             __uint_as_float(sh0.w), __uint_as_float(sh1.x), __uint_as_float(sh1.y),
+                             __uint_as_float(sh1.z), __uint_as_float(sh1.w)};
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        uint32_t a[4], b[4];
-        unpack_signed(w[jj >> 1][(jj & 1) * 2], a);      // row g
-        unpack_signed(w[jj >> 1][(jj & 1) * 2 + 1], b);  // row g + 8
+        for (int jj = 0; jj < 8; ++jj) {
+          uint32_t a[4], b[4];
+          unpack_signed(w[jj >> 1][(jj & 1) * 2], a);      // row g
+          unpack_signed(w[jj >> 1][(jj & 1) * 2 + 1], b);  // row g + 8
 #pragma unroll
-        for (int j = 0; j < kAcc; ++j) {
-          const uint4 xf = (NT == 0 || xok[j]) ? xrow[j][kt * 32 + 4 * jj] : make_uint4(0u, 0u, 0u, 0u);
-          float d[4];
-          mma_first(d, a[0], b[0], a[1], b[1], xf.x, xf.y);
-          mma_next(d, a[2], b[2], a[3], b[3], xf.z, xf.w);
-          acc[j][0] = fmaf(d[0], s0[jj], acc[j][0]);
-          acc[j][2] = fmaf(d[2], s1[jj], acc[j][2]);
-          if (NT != 0) {
-            acc[j][1] = fmaf(d[1], s0[jj], acc[j][1]);
-            acc[j][3] = fmaf(d[3], s1[jj], acc[j][3]);
+          for (int j = 0; j < kAcc; ++j) {
+            const uint4 xf = (NT == 0 || xok[j]) ? xrow[j][kt * 32 + 4 * jj] : make_uint4(0u, 0u, 0u, 0u);
+            float d[4];
+            mma_first(d, a[0], b[0], a[1], b[1], xf.x, xf.y);
+            mma_next(d, a[2], b[2], a[3], b[3], xf.z, xf.w);
+            acc[j][0] = fmaf(d[0], s0[jj], acc[j][0]);
+            acc[j][2] = fmaf(d[2], s1[jj], acc[j][2]);
+            if (NT != 0) {
+              acc[j][1] = fmaf(d[1], s0[jj], acc[j][1]);
+              acc[j][3] = fmaf(d[3], s1[jj], acc[j][3]);
+            }
+          }
+        }
+      } else {
+        // act-order: each chunk's group from the table; (scale, zero) of rows g and g + 8
+        // re-read only when the group changes (consecutive chunks usually share it)
+        const int64_t row_g = row0 + g;
+        int cur = -3;
+        float s0 = 0.0f, s1 = 0.0f;
+        uint32_t zz0 = 0x43004300u, zz1 = 0x43004300u;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c = kt * 8 + jj;
+          const int grp = gtab[c];
+          if (grp == -2) continue;  // past K
+          const uint32_t wg = w[jj >> 1][(jj & 1) * 2], wg8 = w[jj >> 1][(jj & 1) * 2 + 1];
+          if (grp >= 0) {
+            if (grp != cur) {
+              cur = grp;
+              uint32_t z0 = 0u, z1 = 0u;
+              if (p.asym_staged) {
+                // this stage's copy of the row block's scales [16][n_groups] and zeros [16][n_groups]
+                const uint8_t *sa = smem + slot * kStageBytes + kKtilesPerStage * kCodeBox;
+                const float *sc = reinterpret_cast<const float *>(sa);
+                const uint8_t *zr = sa + kRowsPerBlock * p.n_groups * 4;
+                s0 = sc[g * p.n_groups + grp];
+                s1 = sc[(g + 8) * p.n_groups + grp];
+                z0 = static_cast<uint32_t>(zr[g * p.n_groups + grp]) & 15u;
+                z1 = static_cast<uint32_t>(zr[(g + 8) * p.n_groups + grp]) & 15u;
+              } else {
+                s0 = s1 = 0.0f;
+                if (row_g < p.N) {
+                  s0 = __ldg(p.scales + row_g * p.n_groups + grp);
+                  z0 = static_cast<uint32_t>(__ldg(p.zeros + row_g * p.n_groups + grp)) & 15u;
+                }
+                if (row_g + 8 < p.N) {
+                  s1 = __ldg(p.scales + (row_g + 8) * p.n_groups + grp);
+                  z1 = static_cast<uint32_t>(__ldg(p.zeros + (row_g + 8) * p.n_groups + grp)) & 15u;
+                }
+              }
+              zz0 = (0x4300u | z0) * 0x00010001u;
+              zz1 = (0x4300u | z1) * 0x00010001u;
+            }
+            uint32_t a[4], b[4];
+            unpack_asym(wg, zz0, a);
+            unpack_asym(wg8, zz1, b);
+#pragma unroll
+            for (int j = 0; j < kAcc; ++j) {
+              const uint4 xf = (NT == 0 || xok[j]) ? xrow[j][c * 4] : make_uint4(0u, 0u, 0u, 0u);
+              float d[4];
+              mma_first(d, a[0], b[0], a[1], b[1], xf.x, xf.y);
+              mma_next(d, a[2], b[2], a[3], b[3], xf.z, xf.w);
+              acc[j][0] = fmaf(d[0], s0, acc[j][0]);
+              acc[j][2] = fmaf(d[2], s1, acc[j][2]);
+              if (NT != 0) {
+                acc[j][1] = fmaf(d[1], s0, acc[j][1]);
+                acc[j][3] = fmaf(d[3], s1, acc[j][3]);
+              }
+            }
+          } else {
+            // the chunk straddles groups: exact per-column path, pooled over the row's lanes
+            constexpr int MT = NT == 0 ? 1 : 8 * NT;
+            float part[2][MT];
+            mixed_chunk<MT>(p, row_g, c, t, wg, wg8, xs, part);
+            if (NT == 0) {
+              acc[0][0] += part[0][0];
+              acc[0][2] += part[1][0];
+            } else {
+#pragma unroll
+              for (int j = 0; j < kAcc; ++j) {
+                acc[j][0] += part[0][8 * j + 2 * t];
+                acc[j][1] += part[0][8 * j + 2 * t + 1];
+                acc[j][2] += part[1][8 * j + 2 * t];
+                acc[j][3] += part[1][8 * j + 2 * t + 1];
+              }
+            }
           }
         }
       }
@@ -386,17 +584,20 @@ int sm_count_current() {
 
 // Shapes, alignment and the shared-memory plan; *ctas_per_sm is 1 or 2.
 bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_per_sm) {
-  if (lp.M < 1 || lp.M > kMaxM || lp.asym) return false;
+  if (lp.M < 1 || lp.M > kMaxM) return false;
+  if (lp.asym && (lp.perm == nullptr || reinterpret_cast<uintptr_t>(lp.perm) % 16 != 0 || lp.n_groups < 1))
+    return false;  // act-order codes must be sorted by group (w4_asym_prepare)
   if (lp.K % 128 != 0 || lp.N > 0x7fffffffLL) return false;  // TMA: 16-byte row strides, int32 rows
   if (lp.y_dtype != W4_BF16 && lp.y_dtype != W4_F32) return false;
-  const uintptr_t a = reinterpret_cast<uintptr_t>(lp.codes) | reinterpret_cast<uintptr_t>(lp.scales) |
-                      reinterpret_cast<uintptr_t>(lp.x);
+  const uintptr_t a = reinterpret_cast<uintptr_t>(lp.codes) | reinterpret_cast<uintptr_t>(lp.x) |
+                      (lp.asym ? 0 : reinterpret_cast<uintptr_t>(lp.scales));
   if (a % 16 != 0) return false;
   const int64_t KT = (lp.K + 255) / 256;
   const int64_t x_stride = KT * 512 + 64;  // the 64 bytes keep two rows of a lane quad on distinct banks
   const int64_t tok = lp.M == 1 ? 1 : (lp.M <= 8 ? 8 : 16);
   const int64_t red_floats = kWarps * tok * kRowsPerBlock;
-  const int64_t fixed = kAlignSlack + lp.M * x_stride + 2 * red_floats * 4 + kBarBytes;
+  const int64_t gtab_bytes = lp.asym ? KT * 8 * 4 : 0;
+  const int64_t fixed = kAlignSlack + lp.M * x_stride + 2 * red_floats * 4 + gtab_bytes + kBarBytes;
   int64_t S = (kTwoPerSmSmem - fixed) / kStageBytes;
   int per_sm = 2;
   if (S < 4) {  // long rows or many activation rows: one CTA per SM, a deeper ring
@@ -408,6 +609,11 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   q->x = lp.x;
   q->bias = lp.bias;
   q->y = lp.y;
+  q->scales = lp.scales;
+  q->zeros = lp.zeros;
+  q->g_idx = lp.g_idx;
+  q->perm = lp.perm;
+  q->n_groups = lp.n_groups;
   q->N = lp.N;
   q->K = lp.K;
   q->NB = (lp.N + kRowsPerBlock - 1) / kRowsPerBlock;
@@ -421,12 +627,14 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   q->y_dtype = lp.y_dtype;
   q->prefetch = 0;
   q->boxes3d = 0;
+  q->asym_staged = 0;
+  q->x_sorted = 0;
   *smem = static_cast<int>(fixed + S * kStageBytes);
   *ctas_per_sm = per_sm;
   return true;
 }
 
-template <int NT>
+template <int NT, bool ASYM>
 cudaError_t ensure_smem_attr() {
   static std::mutex mu;
   static bool done[64] = {};
@@ -436,17 +644,17 @@ cudaError_t ensure_smem_attr() {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (!done[dev]) {
-    e = cudaFuncSetAttribute(gemv_tma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    e = cudaFuncSetAttribute(gemv_tma_kernel<NT, ASYM>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return e;
     done[dev] = true;
   }
   return cudaSuccess;
 }
 
-template <int NT>
-cudaError_t launch_typed(const CUtensorMap &mc, const CUtensorMap &ms, const TmaGemvParams &q, int smem, int grid,
-                         int32_t *err, cudaStream_t stream) {
-  cudaError_t e = ensure_smem_attr<NT>();
+template <int NT, bool ASYM>
+cudaError_t launch_typed(const CUtensorMap &mc, const CUtensorMap &ms, const CUtensorMap &mz, const TmaGemvParams &q,
+                         int smem, int grid, int32_t *err, cudaStream_t stream) {
+  cudaError_t e = ensure_smem_attr<NT, ASYM>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -458,7 +666,7 @@ cudaError_t launch_typed(const CUtensorMap &mc, const CUtensorMap &ms, const Tma
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_tma_kernel<NT>, mc, ms, q, err);
+  return cudaLaunchKernelEx(&cfg, gemv_tma_kernel<NT, ASYM>, mc, ms, mz, q, err);
 }
 
 }  // namespace
@@ -469,34 +677,68 @@ bool gemv_tma_supports(const LinearParams &p) {
   return make_params(p, &q, &smem, &per_sm) && encode_fn() != nullptr;
 }
 
-cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, int32_t *err, cudaStream_t stream) {
+cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bfloat16 *x_sorted, int32_t *err,
+                            cudaStream_t stream) {
   TmaGemvParams q;
   int smem = 0, per_sm = 1;
   if (!make_params(lp, &q, &smem, &per_sm)) return cudaErrorNotSupported;
   q.prefetch = prefetch ? 1 : 0;
+  if (lp.asym && x_sorted != nullptr) {
+    if (reinterpret_cast<uintptr_t>(x_sorted) % 16 != 0) return cudaErrorInvalidValue;
+    q.x = x_sorted;
+    q.x_sorted = 1;
+  }
   const int64_t P = lp.K / 2, G = lp.K / 32;
   CUtensorMap mc, ms;
-  // 3-D boxes need whole 256-column tiles of codes and whole 1024-column quads of scales in
-  // every row (a box never reaches past a row's end into the next row)
-  q.boxes3d = lp.K % 1024 == 0 &&
-              make_map_3d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, kKtileCodeBytes, lp.N, P / kKtileCodeBytes,
-                          P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, kKtilesPerStage,
-                          CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map_3d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, 32, lp.N, G / 32, G * 4, 128, 32,
-                          kRowsPerBlock, kKtilesPerStage / 4, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!q.boxes3d &&
-      (!make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes, kRowsPerBlock,
-                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-       !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, G, lp.N, G * 4, 32, kRowsPerBlock,
-                    CU_TENSOR_MAP_SWIZZLE_128B)))
-    return cudaErrorInvalidValue;
+  CUtensorMap mz;
+  if (lp.asym) {
+    // codes; with at most 32 groups per row (multiple of 16: 16-byte zero rows) each stage
+    // also carries the row block's scales and zero points, else the kernel reads them per group
+    q.asym_staged = (lp.n_groups == 16 || lp.n_groups == 32) &&
+                    reinterpret_cast<uintptr_t>(lp.scales) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(lp.zeros) % 16 == 0 &&
+                    make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, lp.n_groups, lp.N,
+                                lp.n_groups * 4, lp.n_groups, kRowsPerBlock, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                    make_map_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.zeros, lp.n_groups, lp.N, lp.n_groups,
+                                lp.n_groups, kRowsPerBlock, CU_TENSOR_MAP_SWIZZLE_NONE);
+    q.boxes3d = lp.K % 256 == 0 &&
+                make_map_3d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, kKtileCodeBytes, lp.N, P / kKtileCodeBytes,
+                            P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, kKtilesPerStage,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!q.boxes3d && !make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes,
+                                   kRowsPerBlock, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    if (!q.asym_staged) ms = mz = mc;  // unused
+  } else {
+    // 3-D boxes need whole 256-column tiles of codes and whole 1024-column quads of scales in
+    // every row (a box never reaches past a row's end into the next row)
+    q.boxes3d = lp.K % 1024 == 0 &&
+                make_map_3d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, kKtileCodeBytes, lp.N, P / kKtileCodeBytes,
+                            P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, kKtilesPerStage,
+                            CU_TENSOR_MAP_SWIZZLE_128B) &&
+                make_map_3d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, 32, lp.N, G / 32, G * 4, 128, 32,
+                            kRowsPerBlock, kKtilesPerStage / 4, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!q.boxes3d &&
+        (!make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes, kRowsPerBlock,
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+         !make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, G, lp.N, G * 4, 32, kRowsPerBlock,
+                      CU_TENSOR_MAP_SWIZZLE_128B)))
+      return cudaErrorInvalidValue;
+    mz = ms;  // unused
+  }
   const int64_t slots = static_cast<int64_t>(sm_count_current()) * per_sm;
   const int64_t grid = q.NB < slots ? q.NB : slots;
   q.rb_q = static_cast<int>(q.NB / grid);
   q.rb_r = static_cast<int>(q.NB % grid);
-  if (lp.M == 1) return launch_typed<0>(mc, ms, q, smem, static_cast<int>(grid), err, stream);
-  if (lp.M <= 8) return launch_typed<1>(mc, ms, q, smem, static_cast<int>(grid), err, stream);
-  return launch_typed<2>(mc, ms, q, smem, static_cast<int>(grid), err, stream);
+  const int gi = static_cast<int>(grid);
+  if (lp.asym) {
+    if (lp.M == 1) return launch_typed<0, true>(mc, ms, mz, q, smem, gi, err, stream);
+    if (lp.M <= 8) return launch_typed<1, true>(mc, ms, mz, q, smem, gi, err, stream);
+    return launch_typed<2, true>(mc, ms, mz, q, smem, gi, err, stream);
+  }
+  if (lp.M == 1) return launch_typed<0, false>(mc, ms, mz, q, smem, gi, err, stream);
+  if (lp.M <= 8) return launch_typed<1, false>(mc, ms, mz, q, smem, gi, err, stream);
+  return launch_typed<2, false>(mc, ms, mz, q, smem, gi, err, stream);
 }
 
 }  // namespace w4i

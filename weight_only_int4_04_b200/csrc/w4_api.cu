@@ -71,7 +71,17 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
   }();
   cudaError_t e;
   if (m1_kernel == 0 && w4i::gemv_tma_supports(p)) {
-    e = w4i::launch_gemv_tma(p, g_weight_prefetch.load(std::memory_order_relaxed) != 0, err, stream);
+    // act-order with room in the workspace: gather x into sorted column order once, so that
+    // no CTA of the GEMV has to gather it
+    const __nv_bfloat16 *xs = nullptr;
+    e = cudaSuccess;
+    if (p.asym && workspace != nullptr && workspace_bytes >= w4i::gemm_tc_asym_workspace(p.M, p.K) &&
+        p.K % 8 == 0) {
+      xs = static_cast<const __nv_bfloat16 *>(workspace);
+      e = w4i::launch_gather_x(p.x, p.perm, p.M, p.K, static_cast<__nv_bfloat16 *>(workspace), stream);
+    }
+    if (e == cudaSuccess)
+      e = w4i::launch_gemv_tma(p, g_weight_prefetch.load(std::memory_order_relaxed) != 0, xs, err, stream);
   } else if ((m1_kernel == 0 || m1_kernel == 3) && w4i::gemv_rows_supports(p)) {
     e = w4i::launch_gemv_rows(p, stream);
   } else if (m1_kernel != 2 && w4i::gemv_stream_supports(p)) {
@@ -185,8 +195,10 @@ w4_status w4_linear(const void *x, int64_t M, const uint8_t *codes, const float 
 }
 
 size_t w4_linear_asym_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t n_groups) {
-  // act-order GEMMs above the decode sizes gather x through perm: M * K bf16
-  if (M < kTcMinM || K % 8 != 0 || n_groups % 16 != 0 || M < 1 || K < 1 || N < 1) return 0;
+  // act-order kernels gather x through perm once per call: M * K bf16 (the tensor-core GEMM
+  // above the decode sizes; the decode kernel when K is a multiple of 128)
+  if (M < 1 || K < 1 || N < 1 || n_groups < 1 || K % 8 != 0) return 0;
+  if (M < kTcMinM ? K % 128 != 0 : n_groups % 16 != 0) return 0;
   return w4i::gemm_tc_asym_workspace(M, K);
 }
 

@@ -61,7 +61,12 @@ bool gemv_mma_supports(const LinearParams &p);
 // a TMA stage ring; launched with programmatic stream serialization. `prefetch` lets it
 // stream codes and scales before the previous kernel of the stream has finished (x and y
 // are touched only after it has).
-cudaError_t launch_gemv_tma(const LinearParams &p, bool prefetch, int32_t *err, cudaStream_t stream);
+// Act-order: `x_sorted` (or null) holds x already gathered through perm (launch_gather_x).
+cudaError_t launch_gemv_tma(const LinearParams &p, bool prefetch, const __nv_bfloat16 *x_sorted, int32_t *err,
+                            cudaStream_t stream);
+// xg[m][j] = x[m][perm[j]] for the act-order kernels (K % 8 == 0, 16-byte aligned xg).
+cudaError_t launch_gather_x(const __nv_bfloat16 *x, const int32_t *perm, int64_t M, int64_t K, __nv_bfloat16 *xg,
+                            cudaStream_t stream);
 bool gemv_tma_supports(const LinearParams &p);
 // Tensor-core GEMM (tcgen05, TMA, TMEM) for larger M, aligned rows. The asymmetric
 // act-order variant gathers x through perm into `workspace` (gemm_tc_asym_workspace bytes).
