@@ -260,7 +260,10 @@ def test_linear_zero_rows(w4):
 # ---------------------------------------------------------------------------
 
 DECODE_EDGE_NK = [(1, 128), (16, 256), (17, 384), (33, 640), (2368, 2048), (2400, 2432), (4100, 4096),
-                  (5000, 1152), (300, 14336), (64, 28672)]
+                  (5000, 1152), (300, 14336), (64, 28672),
+                  # K a multiple of 1024 (whole-stage boxes): one row, odd row counts, a row
+                  # count just above two per CTA slot, rows of 4, 12 and 36 k-tiles
+                  (1, 1024), (3, 3072), (593, 1024), (2049, 3072), (7, 9216)]
 
 
 @pytest.mark.parametrize("NK", DECODE_EDGE_NK)
