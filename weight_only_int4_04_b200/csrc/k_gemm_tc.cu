@@ -286,16 +286,28 @@ bool gemm_tc_supports(const LinearParams &p) {
 __global__ void __launch_bounds__(256) gather_x_kernel(const __nv_bfloat16 *__restrict__ x,
                                                        const int32_t *__restrict__ perm, int64_t M, int64_t K,
                                                        __nv_bfloat16 *__restrict__ xg) {
+  // Launched with programmatic stream serialization: the next kernel may launch at once;
+  // x (written by the previous kernel) is read only after grid_dependency_wait, perm (a
+  // weight) before it.
+  grid_launch_dependents();
   const int64_t units = M * (K / 8);
   const uint16_t *xb = reinterpret_cast<const uint16_t *>(x);
+  bool waited = false;
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
        u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t m = u / (K / 8), j0 = (u % (K / 8)) * 8;
+    const int4 p0 = __ldg(reinterpret_cast<const int4 *>(perm + j0));
+    const int4 p1 = __ldg(reinterpret_cast<const int4 *>(perm + j0) + 1);
+    if (!waited) {
+      grid_dependency_wait();
+      waited = true;
+    }
+    const int32_t col[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
     uint32_t v[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t lo = __ldg(xb + m * K + __ldg(perm + j0 + 2 * i));
-      const uint32_t hi = __ldg(xb + m * K + __ldg(perm + j0 + 2 * i + 1));
+      const uint32_t lo = __ldca(xb + m * K + col[2 * i]);
+      const uint32_t hi = __ldca(xb + m * K + col[2 * i + 1]);
       v[i] = lo | (hi << 16);
     }
     *reinterpret_cast<uint4 *>(xg + m * K + j0) = make_uint4(v[0], v[1], v[2], v[3]);
@@ -304,10 +316,19 @@ __global__ void __launch_bounds__(256) gather_x_kernel(const __nv_bfloat16 *__re
 
 cudaError_t launch_gather_x(const __nv_bfloat16 *x, const int32_t *perm, int64_t M, int64_t K, __nv_bfloat16 *xg,
                             cudaStream_t stream) {
+  if (reinterpret_cast<uintptr_t>(perm) % 16 != 0 || K % 8 != 0) return cudaErrorInvalidValue;
   int64_t blocks = (M * (K / 8) + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  gather_x_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, perm, M, K, xg);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gather_x_kernel, x, perm, M, K, xg);
 }
 
 size_t gemm_tc_asym_workspace(int64_t M, int64_t K) {

@@ -57,6 +57,7 @@ constexpr int kMaxSmem = 227 * 1024;
 constexpr int kMaxM = 16;
 constexpr int kBarConsumers = 1;  // named barrier of the consumer warps
 constexpr int kXBatch = 8;        // x chunks in flight per consumer thread (M = 1, K <= 16384 at once)
+constexpr int kGatherChunks = 8;  // act-order, one row gathered in the kernel: K <= 8 * 8 * 256
 
 struct TmaGemvParams {
   const __nv_bfloat16 *x;
@@ -135,6 +136,26 @@ __device__ void mixed_chunk(const TmaGemvParams &p, int64_t row_g, int c, int t,
     }
 }
 
+// Staged act-order scales [16 rows][n_groups] and zero points [16 rows][n_groups] (one TMA box
+// each per stage, n_groups 16 or 32). The boxes are swizzled so that the eight rows a warp's
+// lane quads read for one group fall on distinct banks: scales with the 128-byte (32
+// groups: 128-byte rows) or 64-byte (16 groups) pattern, zero points with the 32-byte
+// pattern (32 groups; 16-byte rows need none). The patterns XOR the 16-byte chunk index with
+// address bits 7 and up of the 1024/512/256-byte aligned box.
+__device__ __forceinline__ float staged_scale(const uint8_t *sa, int n_groups, int r, int j) {
+  const uint32_t off =
+      n_groups == 32 ? static_cast<uint32_t>(r * 128 + ((((j >> 2) ^ (r & 7)) << 4) | ((j & 3) << 2)))
+                     : static_cast<uint32_t>(r * 64 + ((((j >> 2) ^ ((r >> 1) & 3)) << 4) | ((j & 3) << 2)));
+  return *reinterpret_cast<const float *>(sa + off);
+}
+
+__device__ __forceinline__ uint32_t staged_zero(const uint8_t *za, int n_groups, int r, int j) {
+  const uint32_t off = n_groups == 32
+                           ? static_cast<uint32_t>(r * 32 + ((((j >> 4) ^ ((r >> 2) & 1)) << 4) | (j & 15)))
+                           : static_cast<uint32_t>(r * 16 + j);
+  return za[off];
+}
+
 // One code word of unsigned nibbles -> the exact integers u - z (z: the row's zero point
 // of the chunk's group, as the bf16x2 pair (128 + z, 128 + z)).
 __device__ __forceinline__ void unpack_asym(uint32_t w, uint32_t zz, uint32_t (&a)[4]) {
@@ -159,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
   uint8_t *xs = smem + p.S * kStageBytes;
   float *red = reinterpret_cast<float *>(xs + p.M * p.x_stride);
   int32_t *gtab = reinterpret_cast<int32_t *>(red + 2 * p.red_floats);  // ASYM: group of each chunk
-  uint64_t *full = reinterpret_cast<uint64_t *>(gtab + (ASYM ? p.KT * 8 : 0));
+  int32_t *gtab4 = gtab + p.KT * 8;  // ASYM: group of each 128-column half k-tile (-1: several)
+  uint64_t *full = reinterpret_cast<uint64_t *>(gtab + (ASYM ? p.KT * 10 : 0));
   uint64_t *empty = full + kMaxStages;
   uint64_t *x_full = empty + kMaxStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(x_full + 1);
@@ -262,35 +284,51 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
       }
       gtab[c] = gv;
     }
+    for (int h = threadIdx.x; h < p.KT * 2; h += 32 * kWarps) {
+      int gv = -1;
+      const int64_t c0 = 128 * static_cast<int64_t>(h), c1 = c0 + 127;
+      if (c1 < p.K) {
+        // sorted by group: the first and last column decide whether one group spans the block
+        const int g0 = __ldg(p.g_idx + __ldg(p.perm + c0));
+        if (g0 == __ldg(p.g_idx + __ldg(p.perm + c1))) gv = g0;
+      }
+      gtab4[h] = gv;
+    }
   }
   if (ASYM && !p.x_sorted) {
-    // x gathered through perm here (without a caller-side gather: every CTA gathers all of x)
+    // one activation row gathered through perm by every CTA (host: M = 1, at most
+    // kGatherChunks chunks per thread): x is copied in coalesced 16-byte pieces into the
+    // activation buffer, each thread gathers its chunks from there into registers (perm, a
+    // weight, is read before the grid dependency), then writes them back in fragment order.
     const int per_row = p.KT * 32, valid = static_cast<int>(p.K / 8);
+    uint4 *xr = reinterpret_cast<uint4 *>(xs);
+    const uint16_t *xh = reinterpret_cast<const uint16_t *>(xs);
     grid_dependency_wait();
-    const uint16_t *xb = reinterpret_cast<const uint16_t *>(p.x);
-    for (int c = threadIdx.x; c < per_row; c += 32 * kWarps) {
-      int32_t col[8];
+    for (int c = threadIdx.x; c < valid; c += 32 * kWarps) xr[c] = __ldcg(reinterpret_cast<const uint4 *>(p.x) + c);
+    named_barrier_sync(kBarConsumers, 32 * kWarps);
+    uint4 v[kGatherChunks];
+#pragma unroll
+    for (int k = 0; k < kGatherChunks; ++k) {
+      const int c = static_cast<int>(threadIdx.x) + k * 32 * kWarps;
+      v[k] = make_uint4(0u, 0u, 0u, 0u);
       if (c < valid) {
         const int4 p0 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c);
         const int4 p1 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c + 1);
-        col[0] = p0.x, col[1] = p0.y, col[2] = p0.z, col[3] = p0.w;
-        col[4] = p1.x, col[5] = p1.y, col[6] = p1.z, col[7] = p1.w;
+        const uint32_t r0 = xh[p0.x] | (static_cast<uint32_t>(xh[p0.y]) << 16);
+        const uint32_t r1 = xh[p0.z] | (static_cast<uint32_t>(xh[p0.w]) << 16);
+        const uint32_t r2 = xh[p1.x] | (static_cast<uint32_t>(xh[p1.y]) << 16);
+        const uint32_t r3 = xh[p1.z] | (static_cast<uint32_t>(xh[p1.w]) << 16);
+        v[k].x = prmt(r0, r2, 0x5410);
+        v[k].y = prmt(r0, r2, 0x7632);
+        v[k].z = prmt(r1, r3, 0x5410);
+        v[k].w = prmt(r1, r3, 0x7632);
       }
-      for (int m = 0; m < p.M; ++m) {
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (c < valid) {
-          uint32_t r[4];
+    }
+    named_barrier_sync(kBarConsumers, 32 * kWarps);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            r[i] = static_cast<uint32_t>(__ldcg(xb + m * p.K + col[2 * i])) |
-                   (static_cast<uint32_t>(__ldcg(xb + m * p.K + col[2 * i + 1])) << 16);
-          v.x = prmt(r[0], r[2], 0x5410);
-          v.y = prmt(r[0], r[2], 0x7632);
-          v.z = prmt(r[1], r[3], 0x5410);
-          v.w = prmt(r[1], r[3], 0x7632);
-        }
-        reinterpret_cast<uint4 *>(xs + m * p.x_stride)[c] = v;
-      }
+    for (int k = 0; k < kGatherChunks; ++k) {
+      const int c = static_cast<int>(threadIdx.x) + k * 32 * kWarps;
+      if (c < per_row) xr[c] = v[k];
     }
   } else if (NT == 0) {
     // one activation row (already in sorted order for act-order codes): every thread issues
@@ -413,6 +451,57 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
             }
           }
         }
+      } else if (gtab4[2 * kt] >= 0 && gtab4[2 * kt + 1] >= 0) {
+        // act-order, each 128-column half of the k-tile within one group (e.g. groups of
+        // 128 or 256 columns): one (scale, zero point) per half and row, no per-chunk branch
+        const int64_t row_g = row0 + g;
+        float sv[2][2];
+        uint32_t zv[2][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int grp = gtab4[2 * kt + h];
+          uint32_t z0 = 0u, z1 = 0u;
+          if (p.asym_staged) {
+            const uint8_t *sa = smem + slot * kStageBytes + kKtilesPerStage * kCodeBox;
+            const uint8_t *zr = sa + kRowsPerBlock * p.n_groups * 4;
+            sv[h][0] = staged_scale(sa, p.n_groups, g, grp);
+            sv[h][1] = staged_scale(sa, p.n_groups, g + 8, grp);
+            z0 = staged_zero(zr, p.n_groups, g, grp) & 15u;
+            z1 = staged_zero(zr, p.n_groups, g + 8, grp) & 15u;
+          } else {
+            sv[h][0] = sv[h][1] = 0.0f;
+            if (row_g < p.N) {
+              sv[h][0] = __ldg(p.scales + row_g * p.n_groups + grp);
+              z0 = static_cast<uint32_t>(__ldg(p.zeros + row_g * p.n_groups + grp)) & 15u;
+            }
+            if (row_g + 8 < p.N) {
+              sv[h][1] = __ldg(p.scales + (row_g + 8) * p.n_groups + grp);
+              z1 = static_cast<uint32_t>(__ldg(p.zeros + (row_g + 8) * p.n_groups + grp)) & 15u;
+            }
+          }
+          zv[h][0] = (0x4300u | z0) * 0x00010001u;
+          zv[h][1] = (0x4300u | z1) * 0x00010001u;
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int h = jj >> 2;
+          uint32_t a[4], b[4];
+          unpack_asym(w[jj >> 1][(jj & 1) * 2], zv[h][0], a);
+          unpack_asym(w[jj >> 1][(jj & 1) * 2 + 1], zv[h][1], b);
+#pragma unroll
+          for (int j = 0; j < kAcc; ++j) {
+            const uint4 xf = (NT == 0 || xok[j]) ? xrow[j][kt * 32 + 4 * jj] : make_uint4(0u, 0u, 0u, 0u);
+            float d[4];
+            mma_first(d, a[0], b[0], a[1], b[1], xf.x, xf.y);
+            mma_next(d, a[2], b[2], a[3], b[3], xf.z, xf.w);
+            acc[j][0] = fmaf(d[0], sv[h][0], acc[j][0]);
+            acc[j][2] = fmaf(d[2], sv[h][1], acc[j][2]);
+            if (NT != 0) {
+              acc[j][1] = fmaf(d[1], sv[h][0], acc[j][1]);
+              acc[j][3] = fmaf(d[3], sv[h][1], acc[j][3]);
+            }
+          }
+        }
       } else {
         // act-order: each chunk's group from the table; (scale, zero) of rows g and g + 8
         // re-read only when the group changes (consecutive chunks usually share it)
@@ -433,12 +522,11 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
               if (p.asym_staged) {
                 // this stage's copy of the row block's scales [16][n_groups] and zeros [16][n_groups]
                 const uint8_t *sa = smem + slot * kStageBytes + kKtilesPerStage * kCodeBox;
-                const float *sc = reinterpret_cast<const float *>(sa);
                 const uint8_t *zr = sa + kRowsPerBlock * p.n_groups * 4;
-                s0 = sc[g * p.n_groups + grp];
-                s1 = sc[(g + 8) * p.n_groups + grp];
-                z0 = static_cast<uint32_t>(zr[g * p.n_groups + grp]) & 15u;
-                z1 = static_cast<uint32_t>(zr[(g + 8) * p.n_groups + grp]) & 15u;
+                s0 = staged_scale(sa, p.n_groups, g, grp);
+                s1 = staged_scale(sa, p.n_groups, g + 8, grp);
+                z0 = staged_zero(zr, p.n_groups, g, grp) & 15u;
+                z1 = staged_zero(zr, p.n_groups, g + 8, grp) & 15u;
               } else {
                 s0 = s1 = 0.0f;
                 if (row_g < p.N) {
@@ -565,7 +653,7 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   const int64_t x_stride = KT * 512 + 64;  // the 64 bytes keep two rows of a lane quad on distinct banks
   const int64_t tok = lp.M == 1 ? 1 : (lp.M <= 8 ? 8 : 16);
   const int64_t red_floats = kWarps * tok * kRowsPerBlock;
-  const int64_t gtab_bytes = lp.asym ? KT * 8 * 4 : 0;
+  const int64_t gtab_bytes = lp.asym ? KT * 10 * 4 : 0;
   const int64_t fixed = kAlignSlack + lp.M * x_stride + 2 * red_floats * 4 + gtab_bytes + kBarBytes;
   int64_t S = (kTwoPerSmSmem - fixed) / kStageBytes;
   int per_sm = 2;
@@ -646,6 +734,10 @@ bool gemv_tma_supports(const LinearParams &p) {
   return make_params(p, &q, &smem, &per_sm) && encode_fn() != nullptr;
 }
 
+bool gemv_tma_gathers_x(const LinearParams &p) {
+  return p.asym && p.M == 1 && (p.K + 255) / 256 * 32 <= static_cast<int64_t>(kGatherChunks) * 32 * kWarps;
+}
+
 cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bfloat16 *x_sorted, int32_t *err,
                             cudaStream_t stream) {
   TmaGemvParams q;
@@ -656,6 +748,8 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bf
     if (reinterpret_cast<uintptr_t>(x_sorted) % 16 != 0) return cudaErrorInvalidValue;
     q.x = x_sorted;
     q.x_sorted = 1;
+  } else if (lp.asym && !gemv_tma_gathers_x(lp)) {
+    return cudaErrorInvalidValue;  // several rows (or a long row): x must come gathered
   }
   const int64_t P = lp.K / 2, G = lp.K / 32;
   CUtensorMap mc, ms;
@@ -667,9 +761,11 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bf
                     reinterpret_cast<uintptr_t>(lp.scales) % 16 == 0 &&
                     reinterpret_cast<uintptr_t>(lp.zeros) % 16 == 0 &&
                     make_map_2d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, lp.n_groups, lp.N,
-                                lp.n_groups * 4, lp.n_groups, kRowsPerBlock, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                                lp.n_groups * 4, lp.n_groups, kRowsPerBlock,
+                                lp.n_groups == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B) &&
                     make_map_2d(&mz, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.zeros, lp.n_groups, lp.N, lp.n_groups,
-                                lp.n_groups, kRowsPerBlock, CU_TENSOR_MAP_SWIZZLE_NONE);
+                                lp.n_groups, kRowsPerBlock,
+                                lp.n_groups == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE);
     q.boxes3d = lp.K % 256 == 0 &&
                 make_map_3d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, kKtileCodeBytes, lp.N, P / kKtileCodeBytes,
                             P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, kKtilesPerStage,

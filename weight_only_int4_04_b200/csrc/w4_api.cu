@@ -70,13 +70,16 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
     return 0;
   }();
   cudaError_t e;
-  if (m1_kernel == 0 && w4i::gemv_tma_supports(p)) {
-    // act-order with room in the workspace: gather x into sorted column order once, so that
-    // no CTA of the GEMV has to gather it
+  // act-order beyond one short row: x is gathered into sorted column order once per call,
+  // into the workspace, so that no CTA of the GEMV has to gather it (one row: every CTA
+  // gathers it itself, which costs less than a launch)
+  const bool asym_gather = p.asym && !w4i::gemv_tma_gathers_x(p);
+  const bool ws_gather = workspace != nullptr && workspace_bytes >= w4i::gemm_tc_asym_workspace(p.M, p.K) &&
+                         p.K % 8 == 0;
+  if (m1_kernel == 0 && w4i::gemv_tma_supports(p) && (!asym_gather || ws_gather)) {
     const __nv_bfloat16 *xs = nullptr;
     e = cudaSuccess;
-    if (p.asym && workspace != nullptr && workspace_bytes >= w4i::gemm_tc_asym_workspace(p.M, p.K) &&
-        p.K % 8 == 0) {
+    if (asym_gather) {
       xs = static_cast<const __nv_bfloat16 *>(workspace);
       e = w4i::launch_gather_x(p.x, p.perm, p.M, p.K, static_cast<__nv_bfloat16 *>(workspace), stream);
     }

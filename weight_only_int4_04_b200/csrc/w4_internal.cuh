@@ -68,6 +68,9 @@ cudaError_t launch_gemv_tma(const LinearParams &p, bool prefetch, const __nv_bfl
 cudaError_t launch_gather_x(const __nv_bfloat16 *x, const int32_t *perm, int64_t M, int64_t K, __nv_bfloat16 *xg,
                             cudaStream_t stream);
 bool gemv_tma_supports(const LinearParams &p);
+// Act-order: true when launch_gemv_tma gathers x through perm itself (one activation row of
+// moderate length); otherwise the caller passes x_sorted.
+bool gemv_tma_gathers_x(const LinearParams &p);
 // Tensor-core GEMM (tcgen05, TMA, TMEM) for larger M, aligned rows. The asymmetric
 // act-order variant gathers x through perm into `workspace` (gemm_tc_asym_workspace bytes).
 cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t stream, void *workspace);
