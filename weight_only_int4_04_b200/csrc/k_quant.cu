@@ -11,6 +11,18 @@ namespace {
 
 constexpr int kThreads = 256;
 
+int sm_count() {
+  static int counts[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
 int grid_for(int64_t work_items, int items_per_block) {
   // Enough blocks to cover the work, capped at a multiple of 148 SMs x 8 resident blocks;
   // the kernels are grid-stride loops.
@@ -166,6 +178,83 @@ __global__ void __launch_bounds__(kThreads) dequant_generic_kernel(const uint8_t
   }
 }
 
+// Tile path for widths that are not a multiple of 8 (rows of up to kTileCodeBytes of codes):
+// a CTA owns rows r0 .. r0 + R - 1, whose output is the contiguous flat range
+// [r0 K, (r0 + R) K). Their codes (a contiguous byte range) and scales are copied into
+// shared memory with 16-byte loads; then each thread computes 16-byte aligned chunks of the
+// flat output range straight from shared memory (a chunk may span a row end) and stores
+// them whole; the elements before the first and after the last chunk boundary are stored
+// singly.
+constexpr int kTileCodeBytes = 8 * 1024;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) dequant_tile_kernel(const uint8_t *__restrict__ codes,
+                                                                const float *__restrict__ scales,
+                                                                int64_t N, int64_t K, int rows_per_tile,
+                                                                T *__restrict__ out) {
+  constexpr int kV = 16 / sizeof(T);  // elements per 16-byte chunk
+  extern __shared__ __align__(16) uint8_t dq_smem[];
+  const int64_t P = (K + 1) / 2;
+  const int64_t G = (K + 31) / 32;
+  const int64_t total_code_bytes = N * P;
+  const int code_cap = static_cast<int>((rows_per_tile * P + 31) / 16 * 16);  // bytes of the code tile
+  uint8_t *ct = dq_smem;                                                       // codes, from a 16-byte boundary
+  float *st = reinterpret_cast<float *>(dq_smem + code_cap);                  // scales [R][G]
+  for (int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_tile; r0 < N;
+       r0 += static_cast<int64_t>(gridDim.x) * rows_per_tile) {
+    const int rows = static_cast<int>((N - r0) < rows_per_tile ? (N - r0) : rows_per_tile);
+    // codes: bytes [b0, b1) of the flat code array, fetched as aligned 16-byte words from
+    // the word holding b0 (bytes before b0 land in ct[0 .. lead))
+    const int64_t b0 = r0 * P, b1 = b0 + rows * P;
+    const int64_t w0 = b0 / 16, w1 = (b1 + 15) / 16;
+    const int lead = static_cast<int>(b0 - 16 * w0);
+    const uint4 *cw = reinterpret_cast<const uint4 *>(codes);
+    for (int64_t wi = w0 + threadIdx.x; wi < w1; wi += blockDim.x) {
+      uint4 v;
+      if (16 * (wi + 1) <= total_code_bytes) {
+        v = __ldcs(cw + wi);
+      } else {  // the array's last word, partly past its end
+        __align__(16) uint8_t tmp[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) tmp[i] = (16 * wi + i < total_code_bytes) ? codes[16 * wi + i] : 0;
+        v = *reinterpret_cast<const uint4 *>(tmp);
+      }
+      reinterpret_cast<uint4 *>(ct)[wi - w0] = v;
+    }
+    for (int64_t i = threadIdx.x; i < rows * G; i += blockDim.x) st[i] = __ldg(scales + r0 * G + i);
+    __syncthreads();
+    const int64_t f0 = r0 * K, f1 = f0 + rows * K;  // flat output range
+    auto value = [&](int64_t e) -> T {               // e: element index inside the tile
+      const int64_t i = e / K, k = e - i * K;
+      const uint32_t b = ct[lead + i * P + (k >> 1)];
+      return convert_out<T>(__fmul_rn(signed_nibble(b, static_cast<int>(k & 1)), st[i * G + (k >> 5)]));
+    };
+    const int64_t a0 = (f0 + kV - 1) / kV * kV, a1 = f1 / kV * kV;  // chunk boundaries inside
+    if (a1 > a0) {
+      for (int64_t c = threadIdx.x; c < (a1 - a0) / kV; c += blockDim.x) {
+        const int64_t e0 = a0 - f0 + c * kV;  // below R * K < 2^31
+        int64_t i = static_cast<uint32_t>(e0) / static_cast<uint32_t>(K), k = e0 - i * K;
+        __align__(16) T v[kV];
+#pragma unroll
+        for (int u = 0; u < kV; ++u) {
+          const uint32_t b = ct[lead + i * P + (k >> 1)];
+          v[u] = convert_out<T>(__fmul_rn(signed_nibble(b, static_cast<int>(k & 1)), st[i * G + (k >> 5)]));
+          if (++k == K) {
+            k = 0;
+            ++i;
+          }
+        }
+        __stcs(reinterpret_cast<uint4 *>(out + f0 + e0), *reinterpret_cast<const uint4 *>(v));
+      }
+      if (threadIdx.x < a0 - f0) out[f0 + threadIdx.x] = value(threadIdx.x);
+      if (threadIdx.x < f1 - a1) out[a1 + threadIdx.x] = value(a1 - f0 + threadIdx.x);
+    } else {
+      for (int64_t e = threadIdx.x; e < f1 - f0; e += blockDim.x) out[f0 + e] = value(e);
+    }
+    __syncthreads();
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Content validation (page "loopq/packed_weight.py", validate; asymmetric extras).
 // Each thread ORs the rules it saw broken into a block-shared word; one atomic per block.
@@ -258,6 +347,20 @@ static cudaError_t dequant_typed(const uint8_t *codes, const float *scales, int6
                    (reinterpret_cast<uintptr_t>(out) % 16 == 0);
   if (vec) {
     dequant_vec_kernel<T><<<grid_for(N * (K / 8), kThreads), kThreads, 0, stream>>>(codes, scales, N, K, o);
+  } else if (reinterpret_cast<uintptr_t>(out) % 16 == 0 && reinterpret_cast<uintptr_t>(codes) % 16 == 0 &&
+             (K + 1) / 2 <= kTileCodeBytes) {
+    // rows per tile: at most kTileCodeBytes of codes, and few enough that the tiles fill
+    // one wave of resident blocks
+    const int64_t P = (K + 1) / 2, G = (K + 31) / 32;
+    int64_t rows = kTileCodeBytes / P;
+    const int64_t wave = static_cast<int64_t>(sm_count()) * 8;
+    const int64_t spread = (N + wave - 1) / wave;
+    if (spread < rows) rows = spread;
+    if (rows < 1) rows = 1;
+    const int64_t tiles = (N + rows - 1) / rows;
+    const int blocks = static_cast<int>(tiles < wave ? tiles : wave);
+    const int smem = static_cast<int>((rows * P + 31) / 16 * 16 + rows * G * 4);
+    dequant_tile_kernel<T><<<blocks, kThreads, smem, stream>>>(codes, scales, N, K, static_cast<int>(rows), o);
   } else {
     dequant_generic_kernel<T><<<grid_for(N * ((K + 1) / 2), kThreads), kThreads, 0, stream>>>(codes, scales,
                                                                                            N, K, o);
