@@ -13,12 +13,16 @@
 //   warp 1     allocates 256 TMEM columns; one thread issues 4 tcgen05.mma (K = 16 each)
 //              per K block and commits the stage back to the producer;
 //   warps 2-9  dequantize: thread (row, half) turns 16 code bytes + 1 scale into 32 bf16
-//              weights with LOP3/PRMT and fp32x2 arithmetic and stores them in the
-//              swizzled canonical K-major layout the MMA reads; then, after the last MMA,
-//              the same warps move D out of TMEM (tcgen05.ld), add the bias in fp32, round
-//              to the output dtype and store y.
-// A 4-stage ring of shared-memory stages (54 KB each) overlaps loads, dequantization and
-// MMA. All waits are bounded (see w4_sync.cuh).
+//              weights with LOP3/PRMT and fp32x2 arithmetic and writes them with
+//              tcgen05.st into the A operand's stage in tensor memory (row = TMEM lane,
+//              the warp's own lane quarter); then, after the last MMA, the same warps move
+//              D out of TMEM (tcgen05.ld), add the bias in fp32, round to the output dtype
+//              and store y.
+// The dequantized A operand never touches shared memory (it would cost 4 B of shared-memory
+// traffic per weight, written by the dequant warps and read by the MMA, against 0.5 B of
+// codes): shared memory holds only the TMA stages of x, codes and scales, and TMEM holds D
+// (BN columns) plus one 32-column A slice per stage. A ring of 5 (BN = 256) or 8 (BN = 64)
+// stages overlaps loads, dequantization and MMA. All waits are bounded (see w4_sync.cuh).
 #include <cuda.h>
 
 #include <mutex>
@@ -35,20 +39,19 @@ constexpr int BK = 64;     // K per stage: one 128-byte swizzle row of bf16
 constexpr int kThreads = 320;
 constexpr int kDequantWarp0 = 2;
 
-constexpr int A_BYTES = BM_W * BK * 2;    // 16 KB
 constexpr int C_BYTES = BM_W * (BK / 2);  // 4 KB of codes
 constexpr int S_BYTES = BM_W * 4 * 4;     // 2 KB: 4 scale columns per row
 constexpr int Z_BYTES = BM_W * 16;        // 2 KB: 16 zero-point columns per row (asymmetric)
+constexpr int A_TMEM_COLS = BK / 2;       // one stage of A in TMEM: 64 bf16 per row = 32 columns
 constexpr int kMaxStagesAsym = 512;       // K <= 32768 on the asymmetric path
 
-// Shared-memory plan for BN activation rows per tile (MMA N = BN: 64 for the mid-M range,
-// 256 for prefill); a narrower tile leaves room for a deeper ring.
+// Shared-memory and tensor-memory plan for BN activation rows per tile (MMA N = BN: 64 for
+// the mid-M range, 256 for prefill); a narrower tile leaves room for a deeper ring.
 template <bool ASYM, int BN>
 struct TcLayout {
-  static constexpr int STAGES = BN <= 64 ? 6 : 4;
+  static constexpr int STAGES = BN <= 64 ? 8 : 5;
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_B = 0;
   static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_S = OFF_C + STAGES * C_BYTES;
   static constexpr int OFF_Z = OFF_S + STAGES * S_BYTES;
@@ -56,7 +59,11 @@ struct TcLayout {
   static constexpr int OFF_BAR = OFF_G + (ASYM ? 2 * kMaxStagesAsym : 0);
   static constexpr int SMEM = OFF_BAR + 256 + 1024;  // barriers + 1 KB alignment slack
   static constexpr uint32_t TX = B_BYTES + C_BYTES + S_BYTES + (ASYM ? Z_BYTES : 0);
-  static constexpr uint32_t TMEM_COLS = BN;
+  // D in columns [0, BN), A stage s in [BN + 32 s, BN + 32 s + 32); allocation: power of 2
+  static constexpr uint32_t TMEM_NEED = BN + STAGES * A_TMEM_COLS;
+  static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                        : TMEM_NEED <= 256 ? 256 : 512;
+  static_assert(TMEM_NEED <= 512, "GEMM exceeds the tensor-memory budget");
   static_assert(SMEM <= 227 * 1024, "GEMM exceeds the shared-memory budget");
 };
 
@@ -146,7 +153,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16_f32(BM_W, BN);
-      const uint32_t a_base = smem_u32(smem + L::OFF_A);
       const uint32_t b_base = smem_u32(smem + L::OFF_B);
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % STAGES;
@@ -156,9 +162,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = umma_desc_sw128(a_base + s * A_BYTES + kk * 32);
+          const uint32_t a_tmem = tmem_d + BN + s * A_TMEM_COLS + kk * 8;  // K = 16: 8 columns
           const uint64_t bd = umma_desc_sw128(b_base + s * L::B_BYTES + kk * 32);
-          umma_bf16(tmem_d, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tmem_d, a_tmem, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&empty[s]);
       }
@@ -169,7 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                      // TMEM lane quarter this warp may access
     const int half = (warp - kDequantWarp0) >> 2;  // which 32 of the stage's 64 columns
     const int r = 32 * q + lane;                 // weight row inside the tile
-    const uint32_t a_row = smem_u32(smem + L::OFF_A) + r * 128;
+    // this warp's lane quarter, columns of its half of the stage's 64 K values
+    const uint32_t a_tmem0 = tmem_d + (static_cast<uint32_t>(32 * q) << 16) + BN + 16 * half;
     for (int kb = 0; kb < KB; ++kb) {
       const int s = kb % STAGES;
       const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
@@ -192,21 +199,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         nb2 = neg_bias_pair(z);
       }
       const uint64_t scale2 = (static_cast<uint64_t>(__float_as_uint(sc)) << 32) | __float_as_uint(sc);
+      uint32_t av[16];  // 32 bf16 of this row: K pairs (2c, 2c + 1) in column c
       if (!ASYM || gs >= 0) {
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const uint4 v = dequant_word_bf16(words[t], scale2, xorc, nb2);
-          const uint32_t chunk = static_cast<uint32_t>(4 * half + t) ^ static_cast<uint32_t>(r & 7);
-          st_shared_v4(a_row + s * A_BYTES + chunk * 16, v);
+          av[4 * t] = v.x;
+          av[4 * t + 1] = v.y;
+          av[4 * t + 2] = v.z;
+          av[4 * t + 3] = v.w;
         }
       } else {
         // this K block spans two groups: per-column scale and zero from global memory
         const int64_t n = n0 + r;
-#pragma unroll 1
+#pragma unroll
         for (int t = 0; t < 4; ++t) {
           uint32_t packed[4];
+#pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
             float wv[2];
+#pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int e = 2 * e2 + h2;
               const int64_t col = static_cast<int64_t>(kb) * BK + 32 * half + 8 * t + e;
@@ -220,11 +232,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(packed[e2]) : "f"(wv[1]), "f"(wv[0]));
           }
-          const uint32_t chunk = static_cast<uint32_t>(4 * half + t) ^ static_cast<uint32_t>(r & 7);
-          st_shared_v4(a_row + s * A_BYTES + chunk * 16, make_uint4(packed[0], packed[1], packed[2], packed[3]));
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) av[4 * t + e2] = packed[e2];
         }
       }
-      fence_proxy_async_smem();
+      tmem_st_32x32b_x16(a_tmem0 + s * A_TMEM_COLS, av);
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full_a[s]);
     }
