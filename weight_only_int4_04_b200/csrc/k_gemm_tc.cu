@@ -12,8 +12,9 @@
 //              (128 rows x 4 groups) land on one mbarrier;
 //   warp 1     allocates 256 TMEM columns; one thread issues 4 tcgen05.mma (K = 16 each)
 //              per K block and commits the stage back to the producer;
-//   warps 2-9  dequantize: thread (row, half) turns 16 code bytes + 1 scale into 32 bf16
-//              weights with LOP3/PRMT and fp32x2 arithmetic and writes them with
+//   warps 2-9  dequantize (warps 2-17 for 64-row activation tiles): thread (row, part)
+//              turns 16 (8) code bytes + 1 scale into 32 (16) bf16 weights with LOP3/PRMT
+//              and fp32x2 arithmetic and writes them with
 //              tcgen05.st into the A operand's stage in tensor memory (row = TMEM lane,
 //              the warp's own lane quarter); then, after the last MMA, the same warps move
 //              D out of TMEM (tcgen05.ld), add the bias in fp32, round to the output dtype
@@ -36,8 +37,11 @@ namespace {
 
 constexpr int BM_W = 128;  // weight rows per tile (MMA M)
 constexpr int BK = 64;     // K per stage: one 128-byte swizzle row of bf16
-constexpr int kThreads = 320;
 constexpr int kDequantWarp0 = 2;
+// Dequant (and epilogue) warps: 16 for 64-row activation tiles, where dequantization is the
+// whole cost of a K block and more warps hide its latency; 8 for prefill tiles.
+constexpr int dequant_warps(int BN) { return BN <= 64 ? 16 : 8; }
+constexpr int threads_for(int BN) { return 32 * (kDequantWarp0 + dequant_warps(BN)); }
 
 constexpr int C_BYTES = BM_W * (BK / 2);  // 4 KB of codes
 constexpr int S_BYTES = BM_W * 4 * 4;     // 2 KB: 4 scale columns per row
@@ -82,7 +86,7 @@ struct TcParams {
 };
 
 template <bool ASYM, int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for(BN), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_codes,
                    const __grid_constant__ CUtensorMap tmap_scales, const __grid_constant__ CUtensorMap tmap_zeros,
                    const TcParams p, int32_t *err) {
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_load[s], 1);
-      mbar_init(&full_a[s], 8);  // one arrive per dequant warp
+      mbar_init(&full_a[s], dequant_warps(BN));  // one arrive per dequant warp
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -117,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (ASYM) {
     // scale column of every 64-column K block of the sorted columns (-1: two groups)
-    for (int kb = threadIdx.x; kb < KB; kb += kThreads) {
+    for (int kb = threadIdx.x; kb < KB; kb += blockDim.x) {
       const int64_t c0 = static_cast<int64_t>(kb) * BK;
       const int64_t last = (c0 + BK - 1 < p.K) ? c0 + BK - 1 : p.K - 1;
       const int32_t g0 = __ldg(p.g_idx + __ldg(p.perm + c0));
@@ -172,23 +176,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---- dequantize into the A stages ----
-    const int q = warp & 3;                      // TMEM lane quarter this warp may access
-    const int half = (warp - kDequantWarp0) >> 2;  // which 32 of the stage's 64 columns
-    const int r = 32 * q + lane;                 // weight row inside the tile
-    // this warp's lane quarter, columns of its half of the stage's 64 K values
-    const uint32_t a_tmem0 = tmem_d + (static_cast<uint32_t>(32 * q) << 16) + BN + 16 * half;
+    constexpr int PARTS = dequant_warps(BN) / 4;  // warps per TMEM lane quarter
+    constexpr int CP = BK / PARTS;                 // K columns of a stage per thread (32 or 16)
+    constexpr int NW = CP / 8;                     // code words per thread (4 or 2)
+    const int q = warp & 3;                        // TMEM lane quarter this warp may access
+    const int part = (warp - kDequantWarp0) >> 2;  // which CP of the stage's 64 columns
+    const int r = 32 * q + lane;                   // weight row inside the tile
+    // this warp's lane quarter, columns of its part of the stage's 64 K values
+    const uint32_t a_tmem0 = tmem_d + (static_cast<uint32_t>(32 * q) << 16) + BN + (CP / 2) * part;
     for (int kb = 0; kb < KB; ++kb) {
       const int s = kb % STAGES;
       const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
       mbar_wait(&full_load[s], ph, abort_flag, err);
-      const uint4 cw = *reinterpret_cast<const uint4 *>(smem + L::OFF_C + s * C_BYTES + r * 32 + 16 * half);
-      const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+      uint32_t words[NW];
+      const uint8_t *cp = smem + L::OFF_C + s * C_BYTES + r * 32 + (CP / 2) * part;
+      if constexpr (NW == 4) {
+        const uint4 cw = *reinterpret_cast<const uint4 *>(cp);
+        words[0] = cw.x, words[1] = cw.y, words[2] = cw.z, words[3] = cw.w;
+      } else {
+        const uint2 cw = *reinterpret_cast<const uint2 *>(cp);
+        words[0] = cw.x, words[1] = cw.y;
+      }
       float sc;
       uint32_t xorc = 0x08080808u;
       uint64_t nb2 = neg_bias_pair(8u);
       int gs = 0;
       if (!ASYM) {
-        sc = reinterpret_cast<const float *>(smem + L::OFF_S + s * S_BYTES)[r * 4 + (kb & 1) * 2 + half];
+        sc = reinterpret_cast<const float *>(smem + L::OFF_S + s * S_BYTES)[r * 4 + (kb & 1) * 2 + ((CP * part) >> 5)];
       } else {
         gs = gstage[kb];
         const int gsc = gs < 0 ? 0 : gs;
@@ -199,10 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         nb2 = neg_bias_pair(z);
       }
       const uint64_t scale2 = (static_cast<uint64_t>(__float_as_uint(sc)) << 32) | __float_as_uint(sc);
-      uint32_t av[16];  // 32 bf16 of this row: K pairs (2c, 2c + 1) in column c
+      uint32_t av[4 * NW];  // CP bf16 of this row: K pairs (2c, 2c + 1) in column c
       if (!ASYM || gs >= 0) {
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
+        for (int t = 0; t < NW; ++t) {
           const uint4 v = dequant_word_bf16(words[t], scale2, xorc, nb2);
           av[4 * t] = v.x;
           av[4 * t + 1] = v.y;
@@ -213,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this K block spans two groups: per-column scale and zero from global memory
         const int64_t n = n0 + r;
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
+        for (int t = 0; t < NW; ++t) {
           uint32_t packed[4];
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
@@ -221,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int e = 2 * e2 + h2;
-              const int64_t col = static_cast<int64_t>(kb) * BK + 32 * half + 8 * t + e;
+              const int64_t col = static_cast<int64_t>(kb) * BK + CP * part + 8 * t + e;
               wv[h2] = 0.0f;
               if (n < p.N && col < p.K) {
                 const int64_t gg = __ldg(p.g_idx + __ldg(p.perm + col));
@@ -236,7 +250,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e2 = 0; e2 < 4; ++e2) av[4 * t + e2] = packed[e2];
         }
       }
-      tmem_st_32x32b_x16(a_tmem0 + s * A_TMEM_COLS, av);
+      if constexpr (NW == 4)
+        tmem_st_32x32b_x16(a_tmem0 + s * A_TMEM_COLS, av);
+      else
+        tmem_st_32x32b_x8(a_tmem0 + s * A_TMEM_COLS, av);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -250,13 +267,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t n = n0 + r;
     const float b = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
 #pragma unroll 1
-    for (int c = 0; c < BN / 64; ++c) {
-      const int col0 = (BN / 2) * half + 32 * c;
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(32 * q) << 16) + col0, v);
+    for (int c = 0; c < BN / PARTS / 16; ++c) {
+      const int col0 = (BN / PARTS) * part + 16 * c;
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(tmem_d + (static_cast<uint32_t>(32 * q) << 16) + col0, v);
       if (n < p.N) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
           const int64_t m = m0 + col0 + j;
           if (m < p.M) {
             const float o = __uint_as_float(v[j]) + b;
@@ -367,7 +384,7 @@ cudaError_t launch_typed(dim3 grid, const CUtensorMap &mx, const CUtensorMap &mc
       done[dev] = true;
     }
   }
-  gemm_tc_kernel<ASYM, BN><<<grid, kThreads, L::SMEM, stream>>>(mx, mc, ms, mz, tp, err);
+  gemm_tc_kernel<ASYM, BN><<<grid, threads_for(BN), L::SMEM, stream>>>(mx, mc, ms, mz, tp, err);
   return cudaGetLastError();
 }
 
