@@ -39,14 +39,16 @@ namespace w4i {
 
 namespace {
 
-constexpr int kWarps = 8;                    // consumer warps; warp kWarps is the producer
-constexpr int kThreads = 32 * (kWarps + 1);  // 288
+constexpr int kWarps = 8;  // consumer warps for M = 1 and 9 <= M <= 16 (the producer is one more warp)
 constexpr int kRowsPerBlock = 16;            // one m16 MMA tile of weight rows
 constexpr int kKtileCodeBytes = 128;         // 256 columns = 8 groups per k-tile
-constexpr int kKtilesPerStage = kWarps;      // one k-tile per consumer warp per stage
 constexpr int kCodeBox = kRowsPerBlock * kKtileCodeBytes;  // 2 KB
 constexpr int kScaleBox = kRowsPerBlock * 32 * 4;          // 2 KB: 32 scales = 4 k-tiles per row
-constexpr int kStageBytes = kKtilesPerStage * kCodeBox + 2 * kScaleBox;  // 20 KB
+// Consumer warps per CTA: 16 for 2 <= M <= 8 (one CTA per SM: its activations take the
+// shared memory a second CTA would need, so the warps come from one CTA), else 8. A stage
+// holds one k-tile per consumer warp.
+constexpr int warps_for(int nt) { return nt == 1 ? 16 : kWarps; }
+constexpr int stage_bytes(int w) { return w * kCodeBox + (w / 4) * kScaleBox; }
 constexpr int kMaxStages = 8;
 constexpr int kBarBytes = (2 * kMaxStages + 1) * 8 + 16;
 constexpr int kAlignSlack = 1024;
@@ -169,15 +171,17 @@ __device__ __forceinline__ void unpack_asym(uint32_t w, uint32_t zz, uint32_t (&
 // one per MMA column of each n-tile. ASYM: unsigned codes sorted by group (act-order),
 // per-(row, group) scale and zero point read through a per-CTA group table.
 template <int NT, bool ASYM>
-__global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
+__global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
     gemv_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
                     const __grid_constant__ CUtensorMap tm_zeros, const TmaGemvParams p, int32_t *err) {
+  constexpr int W = warps_for(NT);            // consumer warps = k-tiles per stage
+  constexpr int SB = stage_bytes(W);          // bytes per stage
   constexpr int kTok = NT == 0 ? 1 : 8 * NT;  // token slots of the reduction buffer
   constexpr int kAcc = NT == 0 ? 1 : NT;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // 1024-byte swizzle atoms
-  uint8_t *xs = smem + p.S * kStageBytes;
+  uint8_t *xs = smem + p.S * SB;
   float *red = reinterpret_cast<float *>(xs + p.M * p.x_stride);
   int32_t *gtab = reinterpret_cast<int32_t *>(red + 2 * p.red_floats);  // ASYM: group of each chunk
   int32_t *gtab4 = gtab + p.KT * 8;  // ASYM: group of each 128-column half k-tile (-1: several)
@@ -194,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.S; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kWarps);
+      mbar_init(&empty[i], W);
     }
     mbar_init(x_full, 1);
     *abort_flag = 0;
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
   __syncthreads();
   grid_launch_dependents();
 
-  if (warp == kWarps) {
+  if (warp == W) {
     // ---- producer: one thread issues every TMA box of the CTA's row blocks ----
     if (lane == 0) {
       int slot = 0, kc = 0;
@@ -223,15 +227,15 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
         if (i == total) break;
         if ((NT == 0 || (ASYM && !p.x_sorted)) && i == early && !p.prefetch) grid_dependency_wait();
         if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, err)) break;
-        const int kt0 = kc * kKtilesPerStage;
-        const int nkt = (p.KT - kt0) < kKtilesPerStage ? (p.KT - kt0) : kKtilesPerStage;
+        const int kt0 = kc * W;
+        const int nkt = (p.KT - kt0) < W ? (p.KT - kt0) : W;
         const int nsb = (nkt + 3) / 4;
-        uint8_t *st = smem + slot * kStageBytes;
+        uint8_t *st = smem + slot * SB;
         if (ASYM) {
           // codes, and (staged layout) the row block's scales and zero points of every group
           const uint32_t sz = p.asym_staged ? static_cast<uint32_t>(kRowsPerBlock * p.n_groups * 5) : 0u;
           if (p.boxes3d) {
-            mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(kKtilesPerStage * kCodeBox) + sz);
+            mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(W * kCodeBox) + sz);
             tma_load_3d(st, &tm_codes, 0, row, kt0, &full[slot]);
           } else {
             mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox) + sz);
@@ -239,21 +243,21 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
               tma_load_2d(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot]);
           }
           if (p.asym_staged) {
-            uint8_t *sa = st + kKtilesPerStage * kCodeBox;
+            uint8_t *sa = st + W * kCodeBox;
             tma_load_2d(sa, &tm_scales, 0, row, &full[slot]);
             tma_load_2d(sa + kRowsPerBlock * p.n_groups * 4, &tm_zeros, 0, row, &full[slot]);
           }
         } else if (p.boxes3d) {
           // whole-stage boxes; k-tiles past the row end read as zeros (and count as bytes)
-          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(kStageBytes));
+          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(SB));
           tma_load_3d(st, &tm_codes, 0, row, kt0, &full[slot]);
-          tma_load_3d(st + kKtilesPerStage * kCodeBox, &tm_scales, 0, row, kt0 / 4, &full[slot]);
+          tma_load_3d(st + W * kCodeBox, &tm_scales, 0, row, kt0 / 4, &full[slot]);
         } else {
           mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox + nsb * kScaleBox));
           for (int j = 0; j < nkt; ++j)
             tma_load_2d(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot]);
           for (int b = 0; b < nsb; ++b)
-            tma_load_2d(st + kKtilesPerStage * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
+            tma_load_2d(st + W * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
                         &full[slot]);
         }
         if (++kc == p.SPR) {
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
   if (ASYM) {
     // act-order: the group of every sorted 32-column chunk (-1: the chunk straddles groups;
     // -2: past K). perm and g_idx are weights (constant).
-    for (int c = threadIdx.x; c < p.KT * 8; c += 32 * kWarps) {
+    for (int c = threadIdx.x; c < p.KT * 8; c += 32 * W) {
       int gv = -2;
       if (32 * static_cast<int64_t>(c) < p.K) {
         const int64_t c0 = 32 * static_cast<int64_t>(c);
@@ -284,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
       }
       gtab[c] = gv;
     }
-    for (int h = threadIdx.x; h < p.KT * 2; h += 32 * kWarps) {
+    for (int h = threadIdx.x; h < p.KT * 2; h += 32 * W) {
       int gv = -1;
       const int64_t c0 = 128 * static_cast<int64_t>(h), c1 = c0 + 127;
       if (c1 < p.K) {
@@ -304,12 +308,12 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
     uint4 *xr = reinterpret_cast<uint4 *>(xs);
     const uint16_t *xh = reinterpret_cast<const uint16_t *>(xs);
     grid_dependency_wait();
-    for (int c = threadIdx.x; c < valid; c += 32 * kWarps) xr[c] = __ldcg(reinterpret_cast<const uint4 *>(p.x) + c);
-    named_barrier_sync(kBarConsumers, 32 * kWarps);
+    for (int c = threadIdx.x; c < valid; c += 32 * W) xr[c] = __ldcg(reinterpret_cast<const uint4 *>(p.x) + c);
+    named_barrier_sync(kBarConsumers, 32 * W);
     uint4 v[kGatherChunks];
 #pragma unroll
     for (int k = 0; k < kGatherChunks; ++k) {
-      const int c = static_cast<int>(threadIdx.x) + k * 32 * kWarps;
+      const int c = static_cast<int>(threadIdx.x) + k * 32 * W;
       v[k] = make_uint4(0u, 0u, 0u, 0u);
       if (c < valid) {
         const int4 p0 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c);
@@ -324,10 +328,10 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
         v[k].w = prmt(r1, r3, 0x7632);
       }
     }
-    named_barrier_sync(kBarConsumers, 32 * kWarps);
+    named_barrier_sync(kBarConsumers, 32 * W);
 #pragma unroll
     for (int k = 0; k < kGatherChunks; ++k) {
-      const int c = static_cast<int>(threadIdx.x) + k * 32 * kWarps;
+      const int c = static_cast<int>(threadIdx.x) + k * 32 * W;
       if (c < per_row) xr[c] = v[k];
     }
   } else if (NT == 0) {
@@ -338,16 +342,16 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
     const int per_row = p.KT * 32, valid = static_cast<int>(p.K / 8);
     const uint4 *x4 = reinterpret_cast<const uint4 *>(p.x);
     uint4 *xr = reinterpret_cast<uint4 *>(xs);
-    for (int base = static_cast<int>(threadIdx.x); base < per_row; base += kXBatch * 32 * kWarps) {
+    for (int base = static_cast<int>(threadIdx.x); base < per_row; base += kXBatch * 32 * W) {
       uint4 r4[kXBatch];
 #pragma unroll
       for (int k = 0; k < kXBatch; ++k) {
-        const int c = base + k * 32 * kWarps;
+        const int c = base + k * 32 * W;
         r4[k] = (c < valid) ? __ldcg(x4 + c) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int k = 0; k < kXBatch; ++k) {
-        const int c = base + k * 32 * kWarps;
+        const int c = base + k * 32 * W;
         if (c < per_row) {
           uint4 v;
           v.x = prmt(r4[k].x, r4[k].z, 0x5410);
@@ -364,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
     const int per_row = p.KT * 32, valid = static_cast<int>(p.K / 8);
     for (int m = 0; m < p.M; ++m) {
       uint4 *xr = reinterpret_cast<uint4 *>(xs + m * p.x_stride);
-      for (int c = threadIdx.x; c < per_row; c += 32 * kWarps) {
+      for (int c = threadIdx.x; c < per_row; c += 32 * W) {
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (c < valid) {
           const uint4 r4 = xr[c];
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
       }
     }
   }
-  named_barrier_sync(kBarConsumers, 32 * kWarps);
+  named_barrier_sync(kBarConsumers, 32 * W);
 
   const int g = lane >> 2, t = lane & 3;
   const uint32_t stages0 = smem_u32(smem);
@@ -386,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
   const uint32_t ld_row = static_cast<uint32_t>(((lane & 7) + ((lane >> 3) & 1) * 8) * kKtileCodeBytes);
   const uint32_t ld_xor = static_cast<uint32_t>(lane & 7), ld_hi = static_cast<uint32_t>(lane >> 4);
   // this warp's 8 scales per row: chunks 2(w%4), 2(w%4)+1 of scale box w/4
-  const uint32_t sbox = static_cast<uint32_t>(kKtilesPerStage * kCodeBox + (warp >> 2) * kScaleBox);
+  const uint32_t sbox = static_cast<uint32_t>(W * kCodeBox + (warp >> 2) * kScaleBox);
   const uint32_t sch = static_cast<uint32_t>(2 * (warp & 3));
   const uint32_t s_lo = static_cast<uint32_t>(g * 128) + ((sch ^ g) << 4);
   const uint32_t s_hi = static_cast<uint32_t>(g * 128) + (((sch + 1) ^ g) << 4);
@@ -413,15 +417,15 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
   int64_t row0 = rb_begin * kRowsPerBlock;
   for (int i = 0; i < total; ++i) {
     mbar_wait(&full[slot], phase, abort_flag, err);
-    const int kt = kc * kKtilesPerStage + warp;
+    const int kt = kc * W + warp;
     if (kt < p.KT) {
-      const uint32_t st = stages0 + static_cast<uint32_t>(slot * kStageBytes);
+      const uint32_t st = stages0 + static_cast<uint32_t>(slot * SB);
       const uint32_t cb = st + static_cast<uint32_t>(warp * kCodeBox);
       uint32_t w[4][4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) ldsm_x4(cb + ld_off[q], w[q]);
       if (!ASYM) {
-        const uint8_t *sp = smem + slot * kStageBytes + sbox;
+        const uint8_t *sp = smem + slot * SB + sbox;
         const uint4 sg0 = *reinterpret_cast<const uint4 *>(sp + s_lo);
         const uint4 sg1 = *reinterpret_cast<const uint4 *>(sp + s_hi);
         const uint4 sh0 = *reinterpret_cast<const uint4 *>(sp + 1024 + s_lo);
@@ -462,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
           const int grp = gtab4[2 * kt + h];
           uint32_t z0 = 0u, z1 = 0u;
           if (p.asym_staged) {
-            const uint8_t *sa = smem + slot * kStageBytes + kKtilesPerStage * kCodeBox;
+            const uint8_t *sa = smem + slot * SB + W * kCodeBox;
             const uint8_t *zr = sa + kRowsPerBlock * p.n_groups * 4;
             sv[h][0] = staged_scale(sa, p.n_groups, g, grp);
             sv[h][1] = staged_scale(sa, p.n_groups, g + 8, grp);
@@ -521,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
               uint32_t z0 = 0u, z1 = 0u;
               if (p.asym_staged) {
                 // this stage's copy of the row block's scales [16][n_groups] and zeros [16][n_groups]
-                const uint8_t *sa = smem + slot * kStageBytes + kKtilesPerStage * kCodeBox;
+                const uint8_t *sa = smem + slot * SB + W * kCodeBox;
                 const uint8_t *zr = sa + kRowsPerBlock * p.n_groups * 4;
                 s0 = staged_scale(sa, p.n_groups, g, grp);
                 s1 = staged_scale(sa, p.n_groups, g + 8, grp);
@@ -605,15 +609,15 @@ __global__ void __launch_bounds__(kThreads, NT == 0 ? 2 : 1)
           rw[kRowsPerBlock + g + 8] = acc[j][3];
         }
       }
-      named_barrier_sync(kBarConsumers, 32 * kWarps);
-      if (warp == (rbl & (kWarps - 1))) {
+      named_barrier_sync(kBarConsumers, 32 * W);
+      if (warp == (rbl & (W - 1))) {
         for (int e = lane; e < p.M * kRowsPerBlock; e += 32) {
           const int m = e / kRowsPerBlock, rr = e % kRowsPerBlock;
           const int64_t n = row0 + rr;
           if (n < p.N) {
             float v = 0.0f;
 #pragma unroll
-            for (int w2 = 0; w2 < kWarps; ++w2) v += r[(w2 * kTok + m) * kRowsPerBlock + rr];
+            for (int w2 = 0; w2 < W; ++w2) v += r[(w2 * kTok + m) * kRowsPerBlock + rr];
             store_y(p, m, n, v);
           }
         }
@@ -652,13 +656,15 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   const int64_t KT = (lp.K + 255) / 256;
   const int64_t x_stride = KT * 512 + 64;  // the 64 bytes keep two rows of a lane quad on distinct banks
   const int64_t tok = lp.M == 1 ? 1 : (lp.M <= 8 ? 8 : 16);
-  const int64_t red_floats = kWarps * tok * kRowsPerBlock;
+  const int W = warps_for(lp.M == 1 ? 0 : (lp.M <= 8 ? 1 : 2));
+  const int64_t SB = stage_bytes(W);
+  const int64_t red_floats = W * tok * kRowsPerBlock;
   const int64_t gtab_bytes = lp.asym ? KT * 10 * 4 : 0;
   const int64_t fixed = kAlignSlack + lp.M * x_stride + 2 * red_floats * 4 + gtab_bytes + kBarBytes;
-  int64_t S = (kTwoPerSmSmem - fixed) / kStageBytes;
+  int64_t S = (kTwoPerSmSmem - fixed) / SB;
   int per_sm = 2;
   if (S < 4) {  // long rows or many activation rows: one CTA per SM, a deeper ring
-    S = (kMaxSmem - fixed) / kStageBytes;
+    S = (kMaxSmem - fixed) / SB;
     per_sm = 1;
   }
   if (S > kMaxStages) S = kMaxStages;
@@ -677,7 +683,7 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   if (q->NB >= (int64_t(1) << 31) / 64) return false;
   q->M = static_cast<int>(lp.M);
   q->KT = static_cast<int>(KT);
-  q->SPR = static_cast<int>((KT + kKtilesPerStage - 1) / kKtilesPerStage);
+  q->SPR = static_cast<int>((KT + W - 1) / W);
   q->S = static_cast<int>(S);
   q->x_stride = static_cast<int>(x_stride);
   q->red_floats = static_cast<int>(red_floats);
@@ -686,7 +692,7 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   q->boxes3d = 0;
   q->asym_staged = 0;
   q->x_sorted = 0;
-  *smem = static_cast<int>(fixed + S * kStageBytes);
+  *smem = static_cast<int>(fixed + S * SB);
   *ctas_per_sm = per_sm;
   return true;
 }
@@ -715,7 +721,7 @@ cudaError_t launch_typed(const CUtensorMap &mc, const CUtensorMap &ms, const CUt
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(32 * (warps_for(NT) + 1));
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -752,6 +758,7 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bf
     return cudaErrorInvalidValue;  // several rows (or a long row): x must come gathered
   }
   const int64_t P = lp.K / 2, G = lp.K / 32;
+  const int W = warps_for(lp.M == 1 ? 0 : (lp.M <= 8 ? 1 : 2));  // k-tiles per stage
   CUtensorMap mc, ms;
   CUtensorMap mz;
   if (lp.asym) {
@@ -768,7 +775,7 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bf
                                 lp.n_groups == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE);
     q.boxes3d = lp.K % 256 == 0 &&
                 make_map_3d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, kKtileCodeBytes, lp.N, P / kKtileCodeBytes,
-                            P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, kKtilesPerStage,
+                            P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, W,
                             CU_TENSOR_MAP_SWIZZLE_128B);
     if (!q.boxes3d && !make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes,
                                    kRowsPerBlock, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -779,10 +786,10 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bf
     // every row (a box never reaches past a row's end into the next row)
     q.boxes3d = lp.K % 1024 == 0 &&
                 make_map_3d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, kKtileCodeBytes, lp.N, P / kKtileCodeBytes,
-                            P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, kKtilesPerStage,
+                            P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, W,
                             CU_TENSOR_MAP_SWIZZLE_128B) &&
                 make_map_3d(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lp.scales, 32, lp.N, G / 32, G * 4, 128, 32,
-                            kRowsPerBlock, kKtilesPerStage / 4, CU_TENSOR_MAP_SWIZZLE_128B);
+                            kRowsPerBlock, W / 4, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!q.boxes3d &&
         (!make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes, kRowsPerBlock,
                       CU_TENSOR_MAP_SWIZZLE_128B) ||
