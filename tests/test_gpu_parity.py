@@ -125,7 +125,8 @@ def _compare_dequant(w4, codes, scales, K):
             assert np.array_equal(a.view(np.uint8), np.ascontiguousarray(ref).view(np.uint8)), name
 
 
-@pytest.mark.parametrize("NK", [(1, 1), (3, 5), (64, 33), (9, 64), (5, 1000), (40, 4095), (8, 4096), (3, 100)])
+@pytest.mark.parametrize("NK", [(1, 1), (3, 5), (64, 33), (9, 64), (5, 1000), (40, 4095), (8, 4096), (3, 100),
+                                (129, 4095), (3, 20001)])
 def test_dequant_bit_exact_all_dtypes(w4, NK):
     N, K = NK
     rng = np.random.default_rng(N * 1000 + K)
@@ -158,6 +159,29 @@ def test_dequant_unaligned_output(w4):
     w4.dequantize(dc, ds, 64, torch.bfloat16, out=out)
     ref = O.dequantize(codes, scales, 64, "bf16")
     assert np.array_equal(out.cpu().view(torch.int16).numpy().view(np.uint16), ref)
+
+
+def test_dequant_unaligned_codes(w4):
+    """Codes starting one byte past a 16-byte boundary (odd width) take the generic path."""
+    rng = np.random.default_rng(2)
+    N, K = 7, 99
+    P = (K + 1) // 2
+    codes = rng.integers(0, 256, size=(N, P), dtype=np.uint8)
+    codes[:, -1] &= 0x0F
+    scales = rng.uniform(0.1, 1, size=(N, (K + 31) // 32)).astype(np.float32)
+    buf = torch.zeros(N * P + 1, dtype=torch.uint8, device="cuda")
+    buf[1:] = dev(codes.reshape(-1))
+    dc = buf[1:].view(N, P)
+    assert dc.data_ptr() % 16 == 1
+    ds = dev(scales)
+    for dt, name in ((torch.bfloat16, "bf16"), (torch.float32, "f32")):
+        out = w4.dequantize(dc, ds, K, dt)
+        ref = O.dequantize(codes, scales, K, name)
+        got = out.cpu()
+        if name == "bf16":
+            assert np.array_equal(got.view(torch.int16).numpy().view(np.uint16), ref)
+        else:
+            assert np.array_equal(got.numpy().view(np.uint8), np.ascontiguousarray(ref).view(np.uint8))
 
 
 # ---------------------------------------------------------------------------
@@ -393,7 +417,7 @@ def test_asym_small(w4, prepared, M, NKG):
     _asym_check(w4, c, prepared)
 
 
-@pytest.mark.parametrize("M", [1, 3, 9, 16])
+@pytest.mark.parametrize("M", [1, 3, 9, 16, 33])
 @pytest.mark.parametrize("NK", [(48, 512), (40, 1280)])
 def test_asym_ragged_groups(w4, M, NK):
     """Act-order groups of uneven sizes (g_idx drawn at random, not a permutation of equal
@@ -406,6 +430,14 @@ def test_asym_ragged_groups(w4, M, NK):
     c["n_groups"] = n_groups
     _asym_check(w4, c, prepared=True)
     _asym_check(w4, c, prepared=False)
+
+
+@pytest.mark.parametrize("K", [16384, 16512])
+def test_asym_one_row_long(w4, K):
+    """One activation row at the longest width the decode kernel gathers itself (16384)
+    and just past it (gathered once into the workspace instead)."""
+    c = workloads.asym_case(M=1, N=40, K=K, group=128, seed=K)
+    _asym_check(w4, c, prepared=True)
 
 
 @pytest.mark.parametrize("M", workloads.ASYM_M)

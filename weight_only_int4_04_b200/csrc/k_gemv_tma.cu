@@ -158,13 +158,21 @@ __device__ __forceinline__ uint32_t staged_zero(const uint8_t *za, int n_groups,
   return za[off];
 }
 
-// One code word of unsigned nibbles -> the exact integers u - z (z: the row's zero point
-// of the chunk's group, as the bf16x2 pair (128 + z, 128 + z)).
-__device__ __forceinline__ void unpack_asym(uint32_t w, uint32_t zz, uint32_t (&a)[4]) {
-  a[0] = bf16x2_sub(nib_pair_bf16(w, 0x43004300u), zz);
-  a[1] = bf16x2_sub(nib_pair_bf16(w >> 4, 0x43004300u), zz);
-  a[2] = bf16x2_sub(nib_pair_bf16(w >> 8, 0x43004300u), zz);
-  a[3] = bf16x2_sub(nib_pair_bf16(w >> 12, 0x43004300u), zz);
+// a + c for bf16x2 pairs as one exact FMA (a * 1.0 + c).
+__device__ __forceinline__ uint32_t bf16x2_add1(uint32_t a, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(0x3F803F80u), "r"(c));
+  return d;
+}
+
+// One code word of unsigned nibbles -> the exact integers u - z. nzz is the bf16x2 pair
+// (-(128 + z), -(128 + z)) of the row's zero point z for the chunk's group, formed once per
+// group, so each nibble pair costs one LOP3 (u into the mantissa of 128.0) and one exact FMA.
+__device__ __forceinline__ void unpack_asym(uint32_t w, uint32_t nzz, uint32_t (&a)[4]) {
+  a[0] = bf16x2_add1(nib_pair_bf16(w, 0x43004300u), nzz);
+  a[1] = bf16x2_add1(nib_pair_bf16(w >> 4, 0x43004300u), nzz);
+  a[2] = bf16x2_add1(nib_pair_bf16(w >> 8, 0x43004300u), nzz);
+  a[3] = bf16x2_add1(nib_pair_bf16(w >> 12, 0x43004300u), nzz);
 }
 
 // NT = 0: M = 1, x broadcast to every MMA column. NT = 1, 2: up to 8 NT activation rows,
@@ -307,6 +315,20 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
     const int per_row = p.KT * 32, valid = static_cast<int>(p.K / 8);
     uint4 *xr = reinterpret_cast<uint4 *>(xs);
     const uint16_t *xh = reinterpret_cast<const uint16_t *>(xs);
+    // this thread's column indices (a weight: the first kHoist chunks' are read before the
+    // wait, which covers K <= 4096; longer rows read the rest after it)
+    constexpr int kHoist = 2;
+    int4 pc[kHoist][2];
+#pragma unroll
+    for (int k = 0; k < kHoist; ++k) {
+      const int c = static_cast<int>(threadIdx.x) + k * 32 * W;
+      if (c < valid) {
+        pc[k][0] = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c);
+        pc[k][1] = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c + 1);
+      } else {
+        pc[k][0] = pc[k][1] = make_int4(0, 0, 0, 0);
+      }
+    }
     grid_dependency_wait();
     for (int c = threadIdx.x; c < valid; c += 32 * W) xr[c] = __ldcg(reinterpret_cast<const uint4 *>(p.x) + c);
     named_barrier_sync(kBarConsumers, 32 * W);
@@ -316,8 +338,14 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
       const int c = static_cast<int>(threadIdx.x) + k * 32 * W;
       v[k] = make_uint4(0u, 0u, 0u, 0u);
       if (c < valid) {
-        const int4 p0 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c);
-        const int4 p1 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c + 1);
+        int4 p0, p1;
+        if (k < kHoist) {
+          p0 = pc[k < kHoist ? k : 0][0];
+          p1 = pc[k < kHoist ? k : 0][1];
+        } else {
+          p0 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c);
+          p1 = __ldg(reinterpret_cast<const int4 *>(p.perm) + 2 * c + 1);
+        }
         const uint32_t r0 = xh[p0.x] | (static_cast<uint32_t>(xh[p0.y]) << 16);
         const uint32_t r1 = xh[p0.z] | (static_cast<uint32_t>(xh[p0.w]) << 16);
         const uint32_t r2 = xh[p1.x] | (static_cast<uint32_t>(xh[p1.y]) << 16);
@@ -483,8 +511,8 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
               z1 = static_cast<uint32_t>(__ldg(p.zeros + (row_g + 8) * p.n_groups + grp)) & 15u;
             }
           }
-          zv[h][0] = (0x4300u | z0) * 0x00010001u;
-          zv[h][1] = (0x4300u | z1) * 0x00010001u;
+          zv[h][0] = ((0x4300u | z0) * 0x00010001u) ^ 0x80008000u;  // -(128 + z) pairs
+          zv[h][1] = ((0x4300u | z1) * 0x00010001u) ^ 0x80008000u;
         }
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
@@ -512,7 +540,7 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
         const int64_t row_g = row0 + g;
         int cur = -3;
         float s0 = 0.0f, s1 = 0.0f;
-        uint32_t zz0 = 0x43004300u, zz1 = 0x43004300u;
+        uint32_t zz0 = 0xC300C300u, zz1 = 0xC300C300u;  // -(128 + z) pairs
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const int c = kt * 8 + jj;
@@ -542,8 +570,8 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
                   z1 = static_cast<uint32_t>(__ldg(p.zeros + (row_g + 8) * p.n_groups + grp)) & 15u;
                 }
               }
-              zz0 = (0x4300u | z0) * 0x00010001u;
-              zz1 = (0x4300u | z1) * 0x00010001u;
+              zz0 = ((0x4300u | z0) * 0x00010001u) ^ 0x80008000u;
+              zz1 = ((0x4300u | z1) * 0x00010001u) ^ 0x80008000u;
             }
             uint32_t a[4], b[4];
             unpack_asym(wg, zz0, a);
