@@ -100,3 +100,12 @@ def test_binding_refuses_cpu_tensors(w4):
 
 def test_workspace_query(w4):
     assert w4.workspace_bytes(1, 4096, 4096) >= 0
+
+
+def test_prepared_linear_requires_cuda_tensors():
+    """w4.Linear refuses host tensors (no CPU fallback), before touching the library."""
+    import torch
+
+    import weight_only_int4_04_b200 as w4
+    with pytest.raises(ValueError):
+        w4.Linear(torch.zeros((4, 8), dtype=torch.uint8), torch.ones((4, 1), dtype=torch.float32))

@@ -204,6 +204,31 @@ def _linear_check(w4, c, out_dtype=torch.bfloat16, rows=None):
     return worst
 
 
+@pytest.mark.parametrize("MNK", [(1, 300, 4096), (4, 256, 1000), (8, 2400, 2432), (33, 96, 4096)])
+def test_prepared_linear_matches_linear(w4, MNK):
+    """w4.Linear (weights checked once) computes the same y as w4.linear, bitwise."""
+    M, N, K = MNK
+    c = workloads.linear_case(M * 7 + N + K, M, N, K)
+    codes, scales = oracle_pack(c["W"])
+    dc, ds, db = dev(codes), dev(scales), dev(c["bias"])
+    x = x_dev(c["x_bits"])
+    layer = w4.Linear(dc, ds, db, K=K)
+    for dt in (torch.bfloat16, torch.float32):
+        y1 = w4.linear(x, dc, ds, K, bias=db, out_dtype=dt)
+        y2 = layer(x, out_dtype=dt)
+        out = torch.empty_like(y1)
+        y3 = layer(x, out=out)
+        assert y3.data_ptr() == out.data_ptr()
+        assert torch.equal(y1, y2) and torch.equal(y1, y3)
+    yr, bound = O.linear(c["x"], codes, scales, K, c["bias"])
+    ok, worst = O.check_linear(y_host(layer(x)), yr, bound)
+    assert ok, worst
+    with pytest.raises(ValueError):
+        layer(x.float())
+    with pytest.raises(ValueError):
+        layer(x[:, : K - 1].contiguous())
+
+
 def test_linear_config1(w4):
     _linear_check(w4, workloads.config1())
     _linear_check(w4, workloads.config1(), out_dtype=torch.float32)

@@ -100,11 +100,21 @@ def _check(status: int, where: str):
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # ctypes converts a plain int for a c_void_p argument; no wrapper object per pointer
+    return None if t is None else t.data_ptr()
+
+
+try:
+    _raw_stream = torch._C._cuda_getCurrentRawStream  # the current stream's handle as an int
+except AttributeError:  # pragma: no cover - older torch
+    _raw_stream = None
 
 
 def _stream():
-    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    """Handle of the current device's current CUDA stream."""
+    if _raw_stream is not None:
+        return _raw_stream(torch.cuda.current_device())
+    return torch.cuda.current_stream().cuda_stream
 
 
 def _need_cuda(*ts):
@@ -152,8 +162,19 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, K: int, out_dtype=torc
     return out
 
 
+_WS_BYTES = {}
+
+
 def workspace_bytes(M: int, N: int, K: int) -> int:
-    return int(_load().w4_linear_workspace_bytes(M, N, K))
+    """Workspace the symmetric linear needs for these sizes (a function of the sizes only;
+    cached per size triple)."""
+    key = (M, N, K)
+    v = _WS_BYTES.get(key)
+    if v is None:
+        v = int(_load().w4_linear_workspace_bytes(M, N, K))
+        if len(_WS_BYTES) < 4096:
+            _WS_BYTES[key] = v
+    return v
 
 
 def asym_workspace_bytes(M: int, N: int, K: int, n_groups: int) -> int:
@@ -188,6 +209,49 @@ def linear(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, K: int | 
     _check(_load().w4_linear(_ptr(x), M, _ptr(codes), _ptr(scales), N, K, _ptr(bias), _ptr(out),
                          DTYPES[out.dtype], _ptr(ws), wsb, _stream()), "w4_linear")
     return out
+
+
+class Linear:
+    """A prepared symmetric linear: ``Linear(codes, scales, bias)(x, out)`` computes what
+    ``linear`` does, with the weight-side arguments checked and converted once (a layer
+    called every decode step pays only the per-call part: x and out). The weights are
+    referenced, not copied: keep them alive and unchanged while the object is used."""
+
+    __slots__ = ("codes", "scales", "bias", "N", "K", "_codes_p", "_scales_p", "_bias_p", "_fn")
+
+    def __init__(self, codes: torch.Tensor, scales: torch.Tensor, bias: torch.Tensor | None = None,
+                 K: int | None = None):
+        _need_cuda(codes, scales, bias)
+        if codes.dtype != torch.uint8 or scales.dtype != torch.float32 or codes.dim() != 2 or scales.dim() != 2:
+            raise ValueError("codes must be uint8 [N, ceil(K/2)] and scales float32 [N, ceil(K/32)]")
+        N = codes.shape[0]
+        K = 2 * codes.shape[1] if K is None else K
+        if codes.shape[1] != (K + 1) // 2 or scales.shape != (N, (K + 31) // 32):
+            raise ValueError("codes / scales do not match K")
+        if bias is not None and (bias.dtype != torch.float32 or bias.numel() != N):
+            raise ValueError("bias must be float32 [N]")
+        if workspace_bytes(1, N, K) != 0:
+            raise ValueError("this build's linear needs a workspace; use linear()")
+        self.codes, self.scales, self.bias, self.N, self.K = codes, scales, bias, N, K
+        self._codes_p, self._scales_p = codes.data_ptr(), scales.data_ptr()
+        self._bias_p = None if bias is None else bias.data_ptr()
+        self._fn = _load().w4_linear
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None, out_dtype=torch.bfloat16) -> torch.Tensor:
+        if not (x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.shape[1] == self.K
+                and x.is_contiguous()):
+            raise ValueError("x must be a contiguous bfloat16 CUDA tensor [M, K]")
+        M = x.shape[0]
+        if out is None:
+            out = torch.empty((M, self.N), dtype=out_dtype, device=x.device)
+        elif not (out.is_cuda and out.is_contiguous() and out.dtype in (torch.bfloat16, torch.float32)
+                  and out.numel() == M * self.N):
+            raise ValueError("out must be a contiguous bf16 or fp32 CUDA tensor [M, N]")
+        st = self._fn(x.data_ptr(), M, self._codes_p, self._scales_p, self.N, self.K, self._bias_p, out.data_ptr(),
+                      0 if out.dtype == torch.bfloat16 else 2, None, 0, _stream())
+        if st != 0:
+            raise W4Error(st, "w4_linear")
+        return out
 
 
 def asym_prepare(codes: torch.Tensor, g_idx: torch.Tensor, K: int, n_groups: int):
