@@ -334,6 +334,27 @@ def test_linear_small_m_tensor_core_path(w4, M, NK):
     _linear_check(w4, c, out_dtype=torch.float32)
 
 
+@pytest.mark.parametrize("special", ["tiny", "huge", "subnormal", "none"])
+def test_linear_decode_activation_range(w4, special):
+    """Activations at the edges of the bf16 range on the M = 1 decode path: finer than
+    fp16's subnormal spacing, beyond fp16's range, bf16 subnormals, or none of those."""
+    N, K = 600, 4096
+    c = workloads.linear_case(4242, 1, N, K)
+    codes, scales = oracle_pack(c["W"])
+    xb = c["x_bits"].copy()
+    if special == "tiny":      # 2^-20 * 1.5: exact in bf16, not in fp16
+        xb[0, 17] = np.float32(1.5 * 2.0 ** -20).view(np.uint32) >> 16
+    elif special == "huge":    # 2^17: beyond fp16's largest finite value
+        xb[0, 4000] = np.float32(2.0 ** 17).view(np.uint32) >> 16
+    elif special == "subnormal":
+        xb[0, 100] = 0x0003
+    x = O.bf16_bits_to_f32(xb).astype(np.float64)
+    y = w4.linear(x_dev(xb), dev(codes), dev(scales), K, bias=dev(c["bias"]), out_dtype=torch.float32)
+    yr, bound = O.linear(x, codes, scales, K, c["bias"])
+    ok, worst = O.check_linear(y_host(y), yr, bound)
+    assert ok, worst
+
+
 def test_linear_decode_unaligned_x(w4):
     """x starting 8 bytes past a 16-byte boundary takes another kernel; same result."""
     c = workloads.linear_case(77, 1, 300, 2048)
