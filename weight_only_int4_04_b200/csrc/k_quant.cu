@@ -231,17 +231,38 @@ __global__ void __launch_bounds__(kThreads) dequant_tile_kernel(const uint8_t *_
     };
     const int64_t a0 = (f0 + kV - 1) / kV * kV, a1 = f1 / kV * kV;  // chunk boundaries inside
     if (a1 > a0) {
+      const uint32_t K32 = static_cast<uint32_t>(K), P32 = static_cast<uint32_t>(P), G32 = static_cast<uint32_t>(G);
       for (int64_t c = threadIdx.x; c < (a1 - a0) / kV; c += blockDim.x) {
-        const int64_t e0 = a0 - f0 + c * kV;  // below R * K < 2^31
-        int64_t i = static_cast<uint32_t>(e0) / static_cast<uint32_t>(K), k = e0 - i * K;
+        const uint32_t e0 = static_cast<uint32_t>(a0 - f0 + c * kV);  // below R * K < 2^31
+        const uint32_t i = e0 / K32, k0 = e0 - i * K32;
         __align__(16) T v[kV];
+        if (k0 + kV <= K32) {
+          // the chunk lies in one row: its kV / 2 + 1 code bytes from one 8-byte window of
+          // shared memory, shifted so that bit 0 holds column k0
+          const uint32_t b = lead + i * P32 + (k0 >> 1);
+          const uint32_t* wp = reinterpret_cast<const uint32_t *>(ct + (b & ~3u));
+          uint64_t win = (static_cast<uint64_t>(wp[1]) << 32) | wp[0];
+          win >>= 8 * (b & 3u) + 4 * (k0 & 1u);
+          const float *srow = st + i * G32;
+          const float s0 = srow[k0 >> 5], s1 = srow[(k0 + kV - 1) >> 5];
 #pragma unroll
-        for (int u = 0; u < kV; ++u) {
-          const uint32_t b = ct[lead + i * P + (k >> 1)];
-          v[u] = convert_out<T>(__fmul_rn(signed_nibble(b, static_cast<int>(k & 1)), st[i * G + (k >> 5)]));
-          if (++k == K) {
-            k = 0;
-            ++i;
+          for (int u = 0; u < kV; ++u) {
+            // nibble n of column k0 + u -> the float 2^23 + (n ^ 8), minus 2^23 + 8: exact q
+            const uint32_t bits = lop3_and_xor(static_cast<uint32_t>(win >> (4 * u)), 0xFu, 0x4B000008u);
+            const float q = __uint_as_float(bits) - 8388616.0f;
+            const float sc = ((k0 + u) >> 5) != (k0 >> 5) ? s1 : s0;
+            v[u] = convert_out<T>(__fmul_rn(q, sc));
+          }
+        } else {
+          int64_t ii = i, k = k0;
+#pragma unroll
+          for (int u = 0; u < kV; ++u) {
+            const uint32_t bb = ct[lead + ii * P + (k >> 1)];
+            v[u] = convert_out<T>(__fmul_rn(signed_nibble(bb, static_cast<int>(k & 1)), st[ii * G + (k >> 5)]));
+            if (++k == K) {
+              k = 0;
+              ++ii;
+            }
           }
         }
         __stcs(reinterpret_cast<uint4 *>(out + f0 + e0), *reinterpret_cast<const uint4 *>(v));
@@ -359,7 +380,8 @@ static cudaError_t dequant_typed(const uint8_t *codes, const float *scales, int6
     if (rows < 1) rows = 1;
     const int64_t tiles = (N + rows - 1) / rows;
     const int blocks = static_cast<int>(tiles < wave ? tiles : wave);
-    const int smem = static_cast<int>((rows * P + 31) / 16 * 16 + rows * G * 4);
+    // + 16: the 8-byte code window of the last chunk may read a few bytes past the tile
+    const int smem = static_cast<int>((rows * P + 31) / 16 * 16 + rows * G * 4 + 16);
     dequant_tile_kernel<T><<<blocks, kThreads, smem, stream>>>(codes, scales, N, K, static_cast<int>(rows), o);
   } else {
     dequant_generic_kernel<T><<<grid_for(N * ((K + 1) / 2), kThreads), kThreads, 0, stream>>>(codes, scales,
