@@ -140,13 +140,22 @@ __global__ void __launch_bounds__(kThreads) dequant_vec_kernel(const uint8_t *__
   const uint32_t *cw = reinterpret_cast<const uint32_t *>(codes);
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = i / words_per_row, q = i % words_per_row;
+    int64_t n, q;
+    if (total <= 0xffffffffLL) {  // 32-bit divide when the index fits (the common case)
+      const uint32_t i32 = static_cast<uint32_t>(i), wpr = static_cast<uint32_t>(words_per_row);
+      n = i32 / wpr;
+      q = i32 - static_cast<uint32_t>(n) * wpr;
+    } else {
+      n = i / words_per_row;
+      q = i % words_per_row;
+    }
     const uint32_t w = __ldcs(cw + i);
     const float s = __ldg(scales + n * G + q / 4);
     __align__(16) T v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float val = signed_nibble((w >> (4 * e)) & 0xFFu, 0);
+      // nibble n -> the float 2^23 + (n ^ 8), minus 2^23 + 8: the exact signed code
+      const float val = __uint_as_float(lop3_and_xor(w >> (4 * e), 0xFu, 0x4B000008u)) - 8388616.0f;
       v[e] = convert_out<T>(__fmul_rn(val, s));
     }
     T *dst = out + n * K + q * 8;
