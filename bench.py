@@ -172,6 +172,25 @@ def run_reference(args):
 # our arm
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest of every rank's `x` (the time of a replicated step is the slowest
+    rank's); `x` itself with a single process. `device`: where the backend's tensors live
+    (a CUDA device for NCCL, the CPU for gloo)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job throughput: the units every replica processed over the slowest rank's time
+    (GB/s for bytes and milliseconds)."""
+    return world * units_per_rank / (ms * 1e-3) / 1e9
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -272,18 +291,14 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
 
     launches = args.steps * len(shapes)
     hbm_peak, tc_peak, tc_sus, peak_kind = peaks()
     # every launch of the timed region is the GEMV kernel: its average duration is the
     # region time per launch (graph launch gaps included, so this is conservative)
     achieved = args.steps * sum(algo_bytes) / (ms * 1e-3) / 1e9
-    value = world * args.steps * step_bytes / (ms * 1e-3) / 1e9
+    value = job_value(args.steps * step_bytes, world, ms)
 
     # per-shape split, measured the same way on graphs of one shape (reported, not timed region)
     per_shape_us = {}
@@ -341,12 +356,8 @@ def main():
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * e2e_steps * step_bytes / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_value = job_value(e2e_steps * step_bytes, world, e2e_ms)
 
     detail = None
     if rank == 0 and not args.no_detail:
