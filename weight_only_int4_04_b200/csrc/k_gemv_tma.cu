@@ -6,7 +6,10 @@
 //   * one or two CTAs per SM (two when their shared memory fits), each owning a balanced
 //     contiguous range of 16-row blocks; a single producer thread walks them in (row block,
 //     2048-column chunk) order and fills a ring of 20 KB shared-memory stages with TMA boxes
-//     of codes and scales, all with the 128-byte swizzle (conflict-free reads below);
+//     of codes and scales, all with the 128-byte swizzle (conflict-free reads below). The
+//     boxes carry the L2 evict-first policy: weights are read once per call, so they should
+//     not push the activations (this call's x, the next call's input) out of L2 -- an x
+//     that has to come back from HBM behind the weight stream costs ~1 us per launch;
 //   * eight consumer warps take one 256-column k-tile of each stage. Per 32-column group a
 //     lane holds one code word of row g and one of row g + 8 (ldmatrix.x4 fetches four such
 //     words, two groups, in one instruction); LOP3 drops each nibble pair into the mantissa
@@ -218,6 +221,7 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
   if (warp == W) {
     // ---- producer: one thread issues every TMA box of the CTA's row blocks ----
     if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
       int slot = 0, kc = 0;
       uint32_t phase = 0;
       int32_t row = static_cast<int32_t>(rb_begin * kRowsPerBlock);
@@ -244,29 +248,29 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
           const uint32_t sz = p.asym_staged ? static_cast<uint32_t>(kRowsPerBlock * p.n_groups * 5) : 0u;
           if (p.boxes3d) {
             mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(W * kCodeBox) + sz);
-            tma_load_3d(st, &tm_codes, 0, row, kt0, &full[slot]);
+            tma_load_3d_hint(st, &tm_codes, 0, row, kt0, &full[slot], pol);
           } else {
             mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox) + sz);
             for (int j = 0; j < nkt; ++j)
-              tma_load_2d(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot]);
+              tma_load_2d_hint(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot], pol);
           }
           if (p.asym_staged) {
             uint8_t *sa = st + W * kCodeBox;
-            tma_load_2d(sa, &tm_scales, 0, row, &full[slot]);
-            tma_load_2d(sa + kRowsPerBlock * p.n_groups * 4, &tm_zeros, 0, row, &full[slot]);
+            tma_load_2d_hint(sa, &tm_scales, 0, row, &full[slot], pol);
+            tma_load_2d_hint(sa + kRowsPerBlock * p.n_groups * 4, &tm_zeros, 0, row, &full[slot], pol);
           }
         } else if (p.boxes3d) {
           // whole-stage boxes; k-tiles past the row end read as zeros (and count as bytes)
           mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(SB));
-          tma_load_3d(st, &tm_codes, 0, row, kt0, &full[slot]);
-          tma_load_3d(st + W * kCodeBox, &tm_scales, 0, row, kt0 / 4, &full[slot]);
+          tma_load_3d_hint(st, &tm_codes, 0, row, kt0, &full[slot], pol);
+          tma_load_3d_hint(st + W * kCodeBox, &tm_scales, 0, row, kt0 / 4, &full[slot], pol);
         } else {
           mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox + nsb * kScaleBox));
           for (int j = 0; j < nkt; ++j)
-            tma_load_2d(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot]);
+            tma_load_2d_hint(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot], pol);
           for (int b = 0; b < nsb; ++b)
-            tma_load_2d(st + W * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
-                        &full[slot]);
+            tma_load_2d_hint(st + W * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
+                        &full[slot], pol);
         }
         if (++kc == p.SPR) {
           kc = 0;

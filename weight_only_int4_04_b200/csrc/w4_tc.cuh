@@ -30,6 +30,31 @@ __device__ __forceinline__ void tma_load_3d(void *dst_smem, const void *tmap, in
       : "memory");
 }
 
+// L2 policy for data read once (streamed weights): evicted before anything else.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void tma_load_2d_hint(void *dst_smem, const void *tmap, int32_t x, int32_t y,
+                                                 uint64_t *bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3}], [%4], %5;" ::"r"(smem_u32(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_hint(void *dst_smem, const void *tmap, int32_t x, int32_t y, int32_t z,
+                                                 uint64_t *bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, "
+      "%3, %4}], [%5], %6;" ::"r"(smem_u32(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major operand in the 128-byte swizzled canonical
 // layout: rows of 128 bytes (64 bf16), 8-row groups 1024 bytes apart, 16-byte chunks XORed
 // with the row index inside the group. Fields: start address >> 4 in bits [0,14), leading
