@@ -11,6 +11,10 @@ examples, closed forms, invariants and brute force.
 Functions whose parity has no independent pin say so in their docstring
 ("parity unpinned"): only ``quantize_asym_minmax``, which exists to shape
 synthetic input data for the asymmetric variant.
+
+``oracle.q4_0`` restates the GGUF Q4_0 block format (32 elements in 18 bytes: a
+binary16 scale, then 16 bytes of 4-bit codes) and its linear, pinned in
+``tests/test_q4_0_oracle.py``.
 """
 
 from .w4_oracle import (  # noqa: F401

@@ -141,3 +141,29 @@ def asym_random_codes(M: int, N: int = ASYM_SHAPE[0], K: int = ASYM_SHAPE[1], gr
     g_idx, perm = draw_act_order(rng, K, group)
     return {"codes": codes, "zeros": zeros, "scales": scales, "x_bits": x_bits, "x": x, "bias": b,
             "g_idx": g_idx, "n_groups": n_groups, "M": M, "N": N, "K": K}
+
+
+Q4_0_SHAPES = DECODE_SHAPES
+"""(N, K) of the GGUF Q4_0 decode GEMVs (the same decoder projections)."""
+
+
+def draw_q4_0_blocks(rng: np.random.Generator, N: int, K: int, d_sigma: float = 0.0056) -> np.ndarray:
+    """Raw GGUF Q4_0 blocks, uint8 ``[N, K/32, 18]`` (K a multiple of 32): per block a
+    binary16 scale ~ N(0, d_sigma^2) (both signs; the default is the size of a block scale
+    of N(0, 0.02^2) weights), stored little-endian in bytes 0-1, then 16 code bytes drawn
+    uniformly from [0, 255]. Only random draws and their storage layout, no arithmetic of
+    the format."""
+    G = K // 32
+    d = (rng.standard_normal((N, G), dtype=np.float32) * np.float32(d_sigma)).astype("<f2")
+    codes = rng.integers(0, 256, size=(N, G, 16), dtype=np.uint8)
+    dbytes = np.ascontiguousarray(d).view(np.uint8).reshape(N, G, 2)
+    return np.ascontiguousarray(np.concatenate([dbytes, codes], axis=2))
+
+
+def q4_0_case(seed, M: int, N: int, K: int, bias: bool = True):
+    """A Q4_0 linear case: dict with blocks, x_bits, x, bias (or None)."""
+    rng = np.random.default_rng([1, int(seed)])
+    blocks = draw_q4_0_blocks(rng, N, K)
+    x_bits, x = draw_x(rng, M, K)
+    b = draw_bias(rng, N) if bias else None
+    return {"blocks": blocks, "x_bits": x_bits, "x": x, "bias": b, "M": M, "N": N, "K": K}
