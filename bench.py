@@ -496,7 +496,25 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
                                 "tflops": fl / us / 1e6})
         return make
 
-    w = {"dequant_4096x4095_bf16": dequant_odd, "quantize_14336x4096": quantize}
+    def q4_0_decode():
+        # the headline's decode step on GGUF Q4_0 blocks (18 bytes per 32 weights): one call
+        # = the three projections in turn, each on its own rotating block copy
+        sets, xs, ys, nb = [], [], [], 0
+        for N, K in workloads.Q4_0_SHAPES:
+            c = workloads.q4_0_case(N + K, 1, N, K, bias=False)
+            blk = torch.from_numpy(c["blocks"]).to(dev)
+            sets.append([blk.clone() for _ in range(ROTATE)])
+            xs.append(bf16(c["x_bits"]))
+            ys.append(torch.empty((1, N), dtype=torch.bfloat16, device=dev))
+            nb += N * (K // 32) * 18
+
+        def step(r):
+            for j in range(len(xs)):
+                w4.linear_q4_0(xs[j], sets[j][r], out=ys[j])
+        return ([lambda r=r: step(r) for r in range(ROTATE)],
+                lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
+
+    w = {"dequant_4096x4095_bf16": dequant_odd, "quantize_14336x4096": quantize, "q4_0_decode_M1_step": q4_0_decode}
     for M in workloads.BATCHED_M:
         w[f"batched_M{M}_14336x4096"] = batched(M)
     for M, N, K in workloads.PREFILL_SHAPES:

@@ -205,6 +205,44 @@ w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8
                            w4_stream_t stream);
 
 /*
+ * GGUF Q4_0 blocks. Page "max/python/max/graph/quantization.py" (Modular MAX),
+ * QuantizationEncoding.Q4_0 and its block parameters: a block encodes 32 consecutive
+ * elements in 2 + 32/2 = 18 bytes, the scale d and then the 4-bit codes. Readings (the page
+ * gives only the sizes and the field order): d is IEEE binary16, little-endian, in bytes
+ * 0-1; code byte j (bytes 2 + j, j < 16) holds element j in its LOW nibble and element
+ * j + 16 in its HIGH nibble; an element's value is fp32(d * (code - 8)) (exact).
+ *   blocks  uint8 [N, K/32, 18], row-major: a row's K/32 blocks are consecutive, rows are
+ *           consecutive (row n starts at byte n * K/32 * 18). K must be a multiple of 32.
+ * The content is not checked: a non-finite d makes its block's elements NaN or infinite,
+ * as the definition gives.
+ */
+
+/*
+ * w4_dequantize_q4_0 -- dense [N, K] weight of out_dtype (bf16 / f16 / f32 / f64) from Q4_0
+ * blocks: fp32(d * (code - 8)), then round to nearest even (bf16, f16; f16 overflows to
+ * infinity past 65504) or widen exactly (f64). Bit-identical to that definition.
+ *   out  [N, K] row-major, written.
+ * Errors: W4_ERR_NULL, W4_ERR_SHAPE (sizes, K not a multiple of 32), W4_ERR_DTYPE,
+ * W4_ERR_CUDA.
+ */
+w4_status w4_dequantize_q4_0(const uint8_t *blocks, int64_t N, int64_t K, w4_dtype out_dtype, void *out,
+                             w4_stream_t stream);
+
+/*
+ * w4_linear_q4_0 -- y = x . dequant(W)^T (+ bias) for Q4_0 blocks, fp32 accumulation:
+ * |y - y_ref| <= 4e-3 * sum_k |x w| + 1e-6 per element (y_ref the exact sum of x times the
+ * fp32 dequantized weight, plus the bias).
+ *   x     bf16 [M, K] row-major.    bias  optional float32 [N].
+ *   y     [M, N] row-major, bf16 or float32 (y_dtype), written.
+ * M = 1 with K a multiple of 256 and 16-byte aligned x and blocks runs the TMA-fed
+ * tensor-core decode GEMV (launched like w4_linear's decode kernel: programmatic dependent
+ * launch, and w4_set_weight_prefetch applies); every other shape a plain kernel.
+ * Errors: W4_ERR_NULL, W4_ERR_SHAPE, W4_ERR_DTYPE (y_dtype not bf16 / f32), W4_ERR_CUDA.
+ */
+w4_status w4_linear_q4_0(const void *x, int64_t M, const uint8_t *blocks, int64_t N, int64_t K,
+                         const float *bias, void *y, w4_dtype y_dtype, w4_stream_t stream);
+
+/*
  * w4_set_weight_prefetch -- launch policy of the decode linear (process-wide; default 0).
  * The source pages have no counterpart to this call: it only decides when a kernel starts.
  * The M = 1 decode kernel is launched with CUDA programmatic dependent launch: it may begin

@@ -109,3 +109,28 @@ def test_prepared_linear_requires_cuda_tensors():
     import weight_only_int4_04_b200 as w4
     with pytest.raises(ValueError):
         w4.Linear(torch.zeros((4, 8), dtype=torch.uint8), torch.ones((4, 1), dtype=torch.float32))
+
+
+def test_q4_0_host_checks(w4):
+    L = w4.lib
+    FAKE = ctypes.c_void_p(0x1000)
+    # NULL pointers, K not a multiple of 32, bad sizes, bad dtypes: rejected before any launch
+    assert L.w4_linear_q4_0(None, 1, FAKE, 4, 64, None, FAKE, 0, None) == 1
+    assert L.w4_linear_q4_0(FAKE, 1, None, 4, 64, None, FAKE, 0, None) == 1
+    assert L.w4_dequantize_q4_0(None, 4, 64, 2, FAKE, None) == 1
+    assert L.w4_linear_q4_0(FAKE, 1, FAKE, 4, 48, None, FAKE, 0, None) == 2
+    assert L.w4_linear_q4_0(FAKE, 0, FAKE, 4, 64, None, FAKE, 0, None) == 2
+    assert L.w4_linear_q4_0(FAKE, 1, FAKE, 0, 64, None, FAKE, 0, None) == 2
+    assert L.w4_dequantize_q4_0(FAKE, 4, 40, 2, FAKE, None) == 2
+    assert L.w4_linear_q4_0(FAKE, 1, FAKE, 4, 64, None, FAKE, 1, None) == 3  # f16 y not offered
+    assert L.w4_dequantize_q4_0(FAKE, 4, 64, 9, FAKE, None) == 3
+
+
+def test_q4_0_binding_refuses_cpu_and_bad_shapes(w4):
+    import torch
+    blocks = torch.zeros((4, 2, 18), dtype=torch.uint8)
+    x = torch.zeros((1, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        w4.linear_q4_0(x, blocks)
+    with pytest.raises(ValueError):
+        w4.dequantize_q4_0(blocks, 64)

@@ -32,6 +32,7 @@ EXPORTS = (
     "w4_quantize_rtn", "w4_dequantize", "w4_linear", "w4_linear_workspace_bytes", "w4_linear_asym_workspace_bytes",
     "w4_asym_prepare", "w4_linear_asym_gidx", "w4_linear_asym_gidx_noalloc", "w4_validate", "w4_validate_asym",
     "w4_set_weight_prefetch", "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
+    "w4_dequantize_q4_0", "w4_linear_q4_0",
 )
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -52,6 +53,8 @@ _SIGS = {
     "w4_last_cuda_error": [],
     "w4_status_string": [_i32],
     "w4_version": [],
+    "w4_dequantize_q4_0": [_vp, _i64, _i64, _i32, _vp, _vp],
+    "w4_linear_q4_0": [_vp, _i64, _vp, _i64, _i64, _vp, _vp, _i32, _vp],
 }
 _lib = None
 
@@ -159,6 +162,47 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, K: int, out_dtype=torc
         out = torch.empty((N, K), dtype=out_dtype, device=codes.device)
     _check(_load().w4_dequantize(_ptr(codes), _ptr(scales), N, K, format_version, DTYPES[out_dtype], _ptr(out),
                              _stream()), "w4_dequantize")
+    return out
+
+
+def _q4_0_shape(blocks: torch.Tensor, K: int) -> int:
+    if blocks.dtype != torch.uint8 or blocks.dim() != 3 or K % 32 != 0 or blocks.shape[1:] != (K // 32, 18):
+        raise ValueError("blocks must be uint8 [N, K/32, 18] with K a multiple of 32")
+    if not blocks.is_contiguous():
+        raise ValueError("blocks must be contiguous")
+    return blocks.shape[0]
+
+
+def dequantize_q4_0(blocks: torch.Tensor, K: int, out_dtype=torch.float32,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """Dense ``[N, K]`` weight of ``out_dtype`` from GGUF Q4_0 blocks (uint8 ``[N, K/32, 18]``)."""
+    _need_cuda(blocks, out)
+    N = _q4_0_shape(blocks, K)
+    if out_dtype not in DTYPES:
+        raise ValueError("unsupported output dtype")
+    if out is None:
+        out = torch.empty((N, K), dtype=out_dtype, device=blocks.device)
+    _check(_load().w4_dequantize_q4_0(_ptr(blocks), N, K, DTYPES[out.dtype], _ptr(out), _stream()),
+           "w4_dequantize_q4_0")
+    return out
+
+
+def linear_q4_0(x: torch.Tensor, blocks: torch.Tensor, bias: torch.Tensor | None = None,
+                out_dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """``y = x . dequant(W)^T + bias`` for GGUF Q4_0 blocks; bf16 ``x [M, K]``, ``y [M, N]``."""
+    _need_cuda(x, blocks, bias, out)
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D bfloat16 tensor")
+    M, K = x.shape
+    N = _q4_0_shape(blocks, K)
+    if bias is not None and (bias.dtype != torch.float32 or bias.numel() != N):
+        raise ValueError("bias must be float32 [N]")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    if out.dtype not in (torch.bfloat16, torch.float32) or out.numel() != M * N or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 or float32 [M, N] tensor")
+    _check(_load().w4_linear_q4_0(_ptr(x), M, _ptr(blocks), N, K, _ptr(bias), _ptr(out), DTYPES[out.dtype],
+                                  _stream()), "w4_linear_q4_0")
     return out
 
 

@@ -303,6 +303,31 @@ w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8
   return W4_OK;
 }
 
+w4_status w4_dequantize_q4_0(const uint8_t *blocks, int64_t N, int64_t K, w4_dtype out_dtype, void *out,
+                             w4_stream_t stream) {
+  if (!blocks || !out) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || K % 32 != 0) return W4_ERR_SHAPE;
+  if (out_dtype != W4_BF16 && out_dtype != W4_F16 && out_dtype != W4_F32 && out_dtype != W4_F64)
+    return W4_ERR_DTYPE;
+  const cudaError_t e =
+      w4i::launch_q4_0_dequantize(blocks, N, K, out_dtype, out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
+}
+
+w4_status w4_linear_q4_0(const void *x, int64_t M, const uint8_t *blocks, int64_t N, int64_t K,
+                         const float *bias, void *y, w4_dtype y_dtype, w4_stream_t stream) {
+  if (!x || !blocks || !y) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || K % 32 != 0 || M < 1 || M > kMaxRows) return W4_ERR_SHAPE;
+  if (y_dtype != W4_BF16 && y_dtype != W4_F32) return W4_ERR_DTYPE;
+  int32_t *err = nullptr;
+  const w4_status st = symbol_ptr(&err, g_device_error);
+  if (st != W4_OK) return st;
+  const cudaError_t e = w4i::launch_q4_0_linear(static_cast<const __nv_bfloat16 *>(x), M, blocks, N, K, bias, y,
+                                                y_dtype, g_weight_prefetch.load(std::memory_order_relaxed) != 0,
+                                                err, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
+}
+
 int w4_set_weight_prefetch(int enable) {
   return g_weight_prefetch.exchange(enable != 0 ? 1 : 0);
 }

@@ -77,6 +77,16 @@ cudaError_t launch_gemm_tc(const LinearParams &p, int32_t *err, cudaStream_t str
 bool gemm_tc_supports(const LinearParams &p);
 size_t gemm_tc_asym_workspace(int64_t M, int64_t K);
 
+// GGUF Q4_0 blocks (uint8 [N, K/32, 18]): the linear (M = 1 with K a multiple of 256 and
+// 16-byte aligned x and blocks on the TMA-fed tensor-core GEMV, anything else on a plain
+// kernel) and the dequantization to a dense [N, K] array of out_dtype.
+cudaError_t launch_q4_0_linear(const __nv_bfloat16 *x, int64_t M, const uint8_t *blocks, int64_t N, int64_t K,
+                               const float *bias, void *y, int y_dtype, bool prefetch, int32_t *err,
+                               cudaStream_t stream);
+bool q4_0_gemv_supports(const void *x, int64_t M, const uint8_t *blocks, int64_t N, int64_t K, int y_dtype);
+cudaError_t launch_q4_0_dequantize(const uint8_t *blocks, int64_t N, int64_t K, int out_dtype, void *out,
+                                   cudaStream_t stream);
+
 // Validation flag bits (w4_validate reports them in the page's order).
 enum : uint32_t {
   FLAG_SCALE = 1u << 0,
