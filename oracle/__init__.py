@@ -27,6 +27,7 @@ from .w4_oracle import (  # noqa: F401
     dequantize_asym_gidx,
     f32_to_bf16_bits,
     linear,
+    linear_backward_x,
     linear_asym_gidx,
     pack_nibbles,
     payload_bytes,

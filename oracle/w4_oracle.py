@@ -229,6 +229,28 @@ def check_linear(y_gpu, y_ref, bound, rtol: float = 4e-3, atol: float = 1e-6):
 
 
 # ---------------------------------------------------------------------------
+# backward of the linear with respect to its input
+# ---------------------------------------------------------------------------
+
+def linear_backward_x(dy, codes, scales, K: int):
+    """Reference for the input gradient ``dx = dy . dequant(W)`` in float64.
+
+    Keras ``_int4_call``'s ``grad_fn`` returns ``matmul(upstream, transpose(float_kernel))``
+    with the kernel stored ``[in, out]``; PaddleNLP ``QuantizationLinearFunc.backward``
+    returns ``matmul(grad_output, qdq_weight.T)``. With the packed weight stored ``[N, K]``
+    (rows = output features) both are ``dx[m, k] = sum_n dy[m, n] * w[n, k]``, ``w`` the
+    exact fp32 dequantized weight (reading: the pages cast it to the compute dtype first;
+    the tolerance covers that rounding). Also ``bound[m, k] = sum_n |dy[m, n] * w[n, k]|``.
+
+    ``dy`` holds the upstream gradient values as fp32 (bf16 gradients widen exactly).
+    Returns ``(dx_ref, bound)``, both float64 ``[M, K]``.
+    """
+    dy64 = np.asarray(dy, dtype=np.float32).astype(np.float64)
+    w64 = dequantize(codes, scales, K, "f32").astype(np.float64)
+    return dy64 @ w64, np.abs(dy64) @ np.abs(w64)
+
+
+# ---------------------------------------------------------------------------
 # a6: asymmetric sub-channel variant with act-order g_idx
 # ---------------------------------------------------------------------------
 
