@@ -514,7 +514,25 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
         return ([lambda r=r: step(r) for r in range(ROTATE)],
                 lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
 
-    w = {"dequant_4096x4095_bf16": dequant_odd, "quantize_14336x4096": quantize, "q4_0_decode_M1_step": q4_0_decode}
+    def backward_x(M):
+        # input gradient dx = dy . dequant(W) of the (14336, 4096) projection
+        def make():
+            N, K = workloads.BATCHED_SHAPE
+            c = workloads.decode_case(N, K, M=1, config=3)
+            codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
+            copies = [(codes.clone(), scales.clone()) for _ in range(ROTATE)]
+            dy_bits, _ = workloads.draw_x(np.random.default_rng([3, M]), M, N)
+            dy = bf16(dy_bits)
+            dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+            need = int(w4.lib.w4_linear_backward_x_workspace_bytes(M, N, K))
+            ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+            nb = payload(N, K) + 2 * M * N + 2 * M * K
+            return ([lambda c=c, s=s: w4.linear_backward_x(dy, c, s, K, out=dx, workspace=ws) for c, s in copies],
+                    lambda us: {"us": us, "gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
+        return make
+
+    w = {"dequant_4096x4095_bf16": dequant_odd, "quantize_14336x4096": quantize, "q4_0_decode_M1_step": q4_0_decode,
+         "backward_x_M1_14336x4096": backward_x(1), "backward_x_M16_14336x4096": backward_x(16)}
     for M in workloads.BATCHED_M:
         w[f"batched_M{M}_14336x4096"] = batched(M)
     for M, N, K in workloads.PREFILL_SHAPES:

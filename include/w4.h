@@ -205,6 +205,29 @@ w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8
                            w4_stream_t stream);
 
 /*
+ * w4_linear_backward_x -- input gradient of w4_linear: dx = dy . dequant(W).
+ * Keras page (keras/src/layers/core/dense.py, int4 diff), _int4_call's grad_fn:
+ * inputs_grad = matmul(upstream, transpose(float_kernel)); PaddleNLP page
+ * (paddlenlp/quantization/quantization_linear.py), QuantizationLinearFunc.backward:
+ * input_grad = matmul(grad_output, qdq_weight.T). With W stored [N, K] as above:
+ *     dx[m][k] = sum_n dy[m][n] * fp32(value[n][k] * scales[n][k/32]),
+ * fp32 accumulation: |dx - dx_ref| <= 4e-3 * sum_n |dy w| + 1e-6 per element.
+ *   dy   bf16 [M, N] row-major (the upstream gradient).   codes, scales: as w4_linear.
+ *   dx   [M, K] row-major, bf16 or float32 (dx_dtype), written.
+ *   workspace  w4_linear_backward_x_workspace_bytes(M, N, K) bytes, 256-byte aligned (0:
+ *        none needed); the rows are split over CTAs and the splits added in a fixed order,
+ *        so results are deterministic.
+ * K a multiple of 8 with 4-byte aligned codes and scales runs the streaming kernel; other
+ * shapes a plain kernel.
+ * Errors: W4_ERR_NULL, W4_ERR_SHAPE, W4_ERR_DTYPE (dx_dtype not bf16 / f32),
+ * W4_ERR_WORKSPACE, W4_ERR_CUDA.
+ */
+size_t w4_linear_backward_x_workspace_bytes(int64_t M, int64_t N, int64_t K);
+w4_status w4_linear_backward_x(const void *dy, int64_t M, const uint8_t *codes, const float *scales, int64_t N,
+                               int64_t K, void *dx, w4_dtype dx_dtype, void *workspace, size_t workspace_bytes,
+                               w4_stream_t stream);
+
+/*
  * GGUF Q4_0 blocks. Page "max/python/max/graph/quantization.py" (Modular MAX),
  * QuantizationEncoding.Q4_0 and its block parameters: a block encodes 32 consecutive
  * elements in 2 + 32/2 = 18 bytes, the scale d and then the 4-bit codes. Readings (the page

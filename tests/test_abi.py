@@ -134,3 +134,15 @@ def test_q4_0_binding_refuses_cpu_and_bad_shapes(w4):
         w4.linear_q4_0(x, blocks)
     with pytest.raises(ValueError):
         w4.dequantize_q4_0(blocks, 64)
+
+
+def test_backward_host_checks(w4):
+    L = w4.lib
+    FAKE = ctypes.c_void_p(0x1000)
+    assert L.w4_linear_backward_x(None, 1, FAKE, FAKE, 4, 64, FAKE, 0, None, 0, None) == 1
+    assert L.w4_linear_backward_x(FAKE, 0, FAKE, FAKE, 4, 64, FAKE, 0, None, 0, None) == 2
+    assert L.w4_linear_backward_x(FAKE, 1, FAKE, FAKE, 4, 64, FAKE, 3, None, 0, None) == 3
+    need = L.w4_linear_backward_x_workspace_bytes(1, 14336, 4096)
+    assert need > 0 and L.w4_linear_backward_x_workspace_bytes(1, 14336, 4096) == need
+    assert L.w4_linear_backward_x(FAKE, 1, FAKE, FAKE, 14336, 4096, FAKE, 0, None, 0, None) == 12
+    assert L.w4_linear_backward_x_workspace_bytes(1, 8, 37) == 0  # plain kernel: none

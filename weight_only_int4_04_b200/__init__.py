@@ -32,7 +32,7 @@ EXPORTS = (
     "w4_quantize_rtn", "w4_dequantize", "w4_linear", "w4_linear_workspace_bytes", "w4_linear_asym_workspace_bytes",
     "w4_asym_prepare", "w4_linear_asym_gidx", "w4_linear_asym_gidx_noalloc", "w4_validate", "w4_validate_asym",
     "w4_set_weight_prefetch", "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
-    "w4_dequantize_q4_0", "w4_linear_q4_0",
+    "w4_dequantize_q4_0", "w4_linear_q4_0", "w4_linear_backward_x_workspace_bytes", "w4_linear_backward_x",
 )
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -55,6 +55,8 @@ _SIGS = {
     "w4_version": [],
     "w4_dequantize_q4_0": [_vp, _i64, _i64, _i32, _vp, _vp],
     "w4_linear_q4_0": [_vp, _i64, _vp, _i64, _i64, _vp, _vp, _i32, _vp],
+    "w4_linear_backward_x_workspace_bytes": [_i64, _i64, _i64],
+    "w4_linear_backward_x": [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _i32, _vp, _sz, _vp],
 }
 _lib = None
 
@@ -74,6 +76,7 @@ def _load():
             f.restype = ctypes.c_int
         handle.w4_linear_workspace_bytes.restype = ctypes.c_size_t
         handle.w4_linear_asym_workspace_bytes.restype = ctypes.c_size_t
+        handle.w4_linear_backward_x_workspace_bytes.restype = ctypes.c_size_t
         handle.w4_status_string.restype = ctypes.c_char_p
         _lib = handle
     return _lib
@@ -252,6 +255,28 @@ def linear(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, K: int | 
     ws, wsb = _workspace(M, N, K, x.device, workspace)
     _check(_load().w4_linear(_ptr(x), M, _ptr(codes), _ptr(scales), N, K, _ptr(bias), _ptr(out),
                          DTYPES[out.dtype], _ptr(ws), wsb, _stream()), "w4_linear")
+    return out
+
+
+def linear_backward_x(dy: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, K: int,
+                      out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Input gradient ``dx = dy . dequant(W)`` of :func:`linear`: bf16 ``dy [M, N]`` ->
+    ``dx [M, K]`` (bf16 or fp32)."""
+    _need_cuda(dy, codes, scales, out, workspace)
+    if dy.dtype != torch.bfloat16 or dy.dim() != 2:
+        raise ValueError("dy must be a 2-D bfloat16 tensor")
+    M, N = dy.shape
+    if codes.shape != (N, (K + 1) // 2) or scales.shape != (N, (K + 31) // 32):
+        raise ValueError("codes / scales do not match dy and K")
+    if out is None:
+        out = torch.empty((M, K), dtype=out_dtype, device=dy.device)
+    if out.dtype not in (torch.bfloat16, torch.float32) or out.numel() != M * K:
+        raise ValueError("out must be a bf16 or float32 [M, K] tensor")
+    need = int(_load().w4_linear_backward_x_workspace_bytes(M, N, K))
+    ws, wsb = _workspace(M, N, K, dy.device, workspace, need=need)
+    _check(_load().w4_linear_backward_x(_ptr(dy), M, _ptr(codes), _ptr(scales), N, K, _ptr(out), DTYPES[out.dtype],
+                                        _ptr(ws), wsb, _stream()), "w4_linear_backward_x")
     return out
 
 

@@ -328,6 +328,25 @@ w4_status w4_linear_q4_0(const void *x, int64_t M, const uint8_t *blocks, int64_
   return e == cudaSuccess ? W4_OK : cuda_fail(e);
 }
 
+size_t w4_linear_backward_x_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return w4i::linear_backward_x_workspace(M, N, K);
+}
+
+w4_status w4_linear_backward_x(const void *dy, int64_t M, const uint8_t *codes, const float *scales, int64_t N,
+                               int64_t K, void *dx, w4_dtype dx_dtype, void *workspace, size_t workspace_bytes,
+                               w4_stream_t stream) {
+  if (!dy || !codes || !scales || !dx) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || M < 1 || M > kMaxRows) return W4_ERR_SHAPE;
+  if (dx_dtype != W4_BF16 && dx_dtype != W4_F32) return W4_ERR_DTYPE;
+  const size_t need = w4i::linear_backward_x_workspace(M, N, K);
+  if (need > 0 && (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256))
+    return W4_ERR_WORKSPACE;
+  const cudaError_t e = w4i::launch_linear_backward_x(static_cast<const __nv_bfloat16 *>(dy), M, codes, scales, N,
+                                                      K, dx, dx_dtype, workspace, workspace_bytes,
+                                                      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
+}
+
 int w4_set_weight_prefetch(int enable) {
   return g_weight_prefetch.exchange(enable != 0 ? 1 : 0);
 }

@@ -87,6 +87,14 @@ bool q4_0_gemv_supports(const void *x, int64_t M, const uint8_t *blocks, int64_t
 cudaError_t launch_q4_0_dequantize(const uint8_t *blocks, int64_t N, int64_t K, int out_dtype, void *out,
                                    cudaStream_t stream);
 
+// Input gradient dx = dy . dequant(W) (symmetric group-32 codes). The fast kernel needs K a
+// multiple of 8 and 4-byte aligned codes and scales, and, when it splits the rows over
+// CTAs, linear_backward_x_workspace(M, N, K) bytes of workspace; otherwise a plain kernel.
+size_t linear_backward_x_workspace(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_linear_backward_x(const __nv_bfloat16 *dy, int64_t M, const uint8_t *codes, const float *scales,
+                                     int64_t N, int64_t K, void *dx, int dx_dtype, void *workspace,
+                                     size_t workspace_bytes, cudaStream_t stream);
+
 // Validation flag bits (w4_validate reports them in the page's order).
 enum : uint32_t {
   FLAG_SCALE = 1u << 0,
