@@ -33,6 +33,8 @@ from .w4_oracle import (  # noqa: F401
     payload_bytes,
     quantize_asym_minmax,
     quantize_rtn,
+    quantize_rtn_channel,
+    expand_channel_scales,
     unpack_signed,
     unpack_unsigned,
     validate,

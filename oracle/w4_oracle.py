@@ -132,6 +132,45 @@ def quantize_rtn(W):
     return q, scales
 
 
+def quantize_rtn_channel(W):
+    """Round-to-nearest symmetric quantization with one fp32 scale per output row.
+
+    Keras ``quantize`` (int4 diff) on its per-channel branch (``block_size`` None or -1)
+    uses ``AbsMaxQuantizer(axis=0, value_range=(-8, 7))``, one scale per output unit
+    (``kernel_scale`` of shape ``(units,)``); the quantizer's body is not on the page.
+    Reading, with the same rule as :func:`quantize_rtn` over the whole row instead of a
+    32-column group and the Keras range:
+
+      amax_n = max_k |w[n, k]|;   s_n = max(fl32(amax_n / 7), FLOOR)
+      q      = clamp(round_half_even(fl32(w / s_n)), -8, 7)
+
+    and the scale multiplies the code (LoopQ's convention; Keras divides by a multiplier
+    ``7 / amax``, the same value up to rounding). With this scale |w / s| <= 7 up to the
+    quotient's rounding, so the codes lie in [-7, 7] and are valid for format v1 too.
+
+    Returns ``(q, scales)``: int8 ``[N, K]`` and fp32 ``[N]``. Raises ValueError for an
+    empty, non-2-D or non-finite W.
+    """
+    W = np.asarray(W)
+    if W.ndim != 2 or min(W.shape) <= 0:
+        raise ValueError("weight must be a nonempty matrix")
+    W = W.astype(np.float32, copy=False)
+    if not np.isfinite(W).all():
+        raise ValueError("weight must be finite")
+    amax = np.max(np.abs(W), axis=1)
+    s = np.maximum(amax / np.float32(QMAX), FLOOR).astype(np.float32)
+    t = (W / s[:, None]).astype(np.float32)
+    q = np.clip(np.rint(t), -8, 7).astype(np.int8)
+    return q, s
+
+
+def expand_channel_scales(scales_channel, K: int) -> np.ndarray:
+    """Per-row scales ``[N]`` as the group layout ``[N, ceil(K/32)]`` (every group of a row
+    carries the row's scale): a per-channel weight is then a packed group-32 weight."""
+    s = np.asarray(scales_channel, dtype=np.float32).reshape(-1, 1)
+    return np.repeat(s, math.ceil(K / GROUP), axis=1)
+
+
 def pack_nibbles(values) -> np.ndarray:
     """Pack 4-bit values two per byte along the width, even column in the low nibble.
 
