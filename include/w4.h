@@ -205,6 +205,30 @@ w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8
                            w4_stream_t stream);
 
 /*
+ * Per-channel symmetric int4: one fp32 scale per output row. Keras page
+ * (keras/src/layers/core/dense.py, int4 diff), quantize's per-channel branch:
+ * AbsMaxQuantizer(axis=0, value_range=(-8, 7)) and kernel_scale of shape (units,); the
+ * quantizer's body is not on the page. Reading, the rule of w4_quantize_rtn over a whole
+ * row and the Keras range: for each row n
+ *     amax = max |W[n][:]|;  s = max(fl32(amax / 7), 2^-126);  q = clamp(rne(fl32(W / s)), -8, 7)
+ * with the codes packed as in the format above (they lie in [-7, 7], valid for v1).
+ * Only the scale layout differs from the group-32 format: w4_expand_channel_scales writes
+ * the row's scale into every group, after which w4_dequantize, w4_linear,
+ * w4_linear_backward_x and w4_validate serve the weight unchanged (keep the expanded array,
+ * as a model keeps its parameters; expanding costs one small kernel).
+ *
+ * w4_quantize_rtn_channel -- W float32 [N, K] -> codes uint8 [N, ceil(K/2)], scales float32
+ *   [N]; d_status as w4_quantize_rtn (NULL: synchronize and return W4_ERR_NONFINITE for a
+ *   non-finite W). Bit-identical to the definition above.
+ * w4_expand_channel_scales -- scales float32 [N] -> scales_out float32 [N, ceil(K/32)].
+ * Errors: W4_ERR_NULL, W4_ERR_SHAPE, W4_ERR_NONFINITE (quantize), W4_ERR_CUDA.
+ */
+w4_status w4_quantize_rtn_channel(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                                  int32_t *d_status, w4_stream_t stream);
+w4_status w4_expand_channel_scales(const float *scales, int64_t N, int64_t K, float *scales_out,
+                                   w4_stream_t stream);
+
+/*
  * w4_linear_backward_x -- input gradient of w4_linear: dx = dy . dequant(W).
  * Keras page (keras/src/layers/core/dense.py, int4 diff), _int4_call's grad_fn:
  * inputs_grad = matmul(upstream, transpose(float_kernel)); PaddleNLP page

@@ -146,3 +146,12 @@ def test_backward_host_checks(w4):
     assert need > 0 and L.w4_linear_backward_x_workspace_bytes(1, 14336, 4096) == need
     assert L.w4_linear_backward_x(FAKE, 1, FAKE, FAKE, 14336, 4096, FAKE, 0, None, 0, None) == 12
     assert L.w4_linear_backward_x_workspace_bytes(1, 8, 37) == 0  # plain kernel: none
+
+
+def test_channel_host_checks(w4):
+    L = w4.lib
+    FAKE = ctypes.c_void_p(0x1000)
+    assert L.w4_quantize_rtn_channel(None, 4, 64, FAKE, FAKE, None, None) == 1
+    assert L.w4_quantize_rtn_channel(FAKE, 0, 64, FAKE, FAKE, None, None) == 2
+    assert L.w4_expand_channel_scales(FAKE, 4, 0, FAKE, None) == 2
+    assert L.w4_expand_channel_scales(None, 4, 64, FAKE, None) == 1

@@ -33,6 +33,7 @@ EXPORTS = (
     "w4_asym_prepare", "w4_linear_asym_gidx", "w4_linear_asym_gidx_noalloc", "w4_validate", "w4_validate_asym",
     "w4_set_weight_prefetch", "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
     "w4_dequantize_q4_0", "w4_linear_q4_0", "w4_linear_backward_x_workspace_bytes", "w4_linear_backward_x",
+    "w4_quantize_rtn_channel", "w4_expand_channel_scales",
 )
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -57,6 +58,8 @@ _SIGS = {
     "w4_linear_q4_0": [_vp, _i64, _vp, _i64, _i64, _vp, _vp, _i32, _vp],
     "w4_linear_backward_x_workspace_bytes": [_i64, _i64, _i64],
     "w4_linear_backward_x": [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _i32, _vp, _sz, _vp],
+    "w4_quantize_rtn_channel": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
+    "w4_expand_channel_scales": [_vp, _i64, _i64, _vp, _vp],
 }
 _lib = None
 
@@ -152,6 +155,31 @@ def quantize_rtn(W: torch.Tensor, status: torch.Tensor | None = None, out=None):
     _check(_load().w4_quantize_rtn(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(status), _stream()),
            "w4_quantize_rtn")
     return codes, scales
+
+
+def quantize_rtn_channel(W: torch.Tensor, status: torch.Tensor | None = None):
+    """Per-channel RTN quantization of fp32 ``W [N, K]`` -> ``(codes uint8 [N, ceil(K/2)],
+    scales float32 [N])``, one scale per row (``status`` as in :func:`quantize_rtn`)."""
+    _need_cuda(W, status)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    N, K = W.shape
+    codes = torch.empty((N, (K + 1) // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _check(_load().w4_quantize_rtn_channel(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(status), _stream()),
+           "w4_quantize_rtn_channel")
+    return codes, scales
+
+
+def expand_channel_scales(scales: torch.Tensor, K: int) -> torch.Tensor:
+    """Per-row scales ``[N]`` -> the group layout ``[N, ceil(K/32)]`` every other call reads."""
+    _need_cuda(scales)
+    if scales.dtype != torch.float32 or scales.dim() != 1:
+        raise ValueError("scales must be a 1-D float32 tensor")
+    N = scales.shape[0]
+    out = torch.empty((N, (K + 31) // 32), dtype=torch.float32, device=scales.device)
+    _check(_load().w4_expand_channel_scales(_ptr(scales), N, K, _ptr(out), _stream()), "w4_expand_channel_scales")
+    return out
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, K: int, out_dtype=torch.float32,

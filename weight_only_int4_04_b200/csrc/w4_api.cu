@@ -347,6 +347,39 @@ w4_status w4_linear_backward_x(const void *dy, int64_t M, const uint8_t *codes, 
   return e == cudaSuccess ? W4_OK : cuda_fail(e);
 }
 
+w4_status w4_quantize_rtn_channel(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                                  int32_t *d_status, w4_stream_t stream) {
+  if (!W || !codes || !scales) return W4_ERR_NULL;
+  if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t *status = d_status;
+  if (!status) {
+    const w4_status st = symbol_ptr(&status, g_quant_status);
+    if (st != W4_OK) return st;
+    const cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  cudaError_t e = w4i::launch_quantize_rtn_channel(W, N, K, codes, scales, status, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!d_status) {
+    int32_t host = 0;
+    e = cudaMemcpyAsync(&host, status, sizeof(host), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (host != 0) return W4_ERR_NONFINITE;
+  }
+  return W4_OK;
+}
+
+w4_status w4_expand_channel_scales(const float *scales, int64_t N, int64_t K, float *scales_out,
+                                   w4_stream_t stream) {
+  if (!scales || !scales_out) return W4_ERR_NULL;
+  if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
+  const cudaError_t e =
+      w4i::launch_expand_channel_scales(scales, N, K, scales_out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
+}
+
 int w4_set_weight_prefetch(int enable) {
   return g_weight_prefetch.exchange(enable != 0 ? 1 : 0);
 }

@@ -95,6 +95,13 @@ cudaError_t launch_linear_backward_x(const __nv_bfloat16 *dy, int64_t M, const u
                                      int64_t N, int64_t K, void *dx, int dx_dtype, void *workspace,
                                      size_t workspace_bytes, cudaStream_t stream);
 
+// Per-channel symmetric int4 (one scale per row): RTN quantize + pack, and the expansion of
+// the [N] scales to the group layout [N, ceil(K/32)] the other kernels read.
+cudaError_t launch_quantize_rtn_channel(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                                        int32_t *status, cudaStream_t stream);
+cudaError_t launch_expand_channel_scales(const float *scales, int64_t N, int64_t K, float *out,
+                                         cudaStream_t stream);
+
 // Validation flag bits (w4_validate reports them in the page's order).
 enum : uint32_t {
   FLAG_SCALE = 1u << 0,
