@@ -28,6 +28,7 @@ from .w4_oracle import (  # noqa: F401
     f32_to_bf16_bits,
     linear,
     linear_backward_x,
+    lora_merge,
     linear_asym_gidx,
     pack_nibbles,
     payload_bytes,

@@ -290,6 +290,40 @@ def linear_backward_x(dy, codes, scales, K: int):
 
 
 # ---------------------------------------------------------------------------
+# LoRA merge: dequantize, add the low-rank update, re-quantize, re-pack
+# ---------------------------------------------------------------------------
+
+def lora_merge(codes, scales, K: int, lora_b_t, lora_a_t, alpha_over_rank):
+    """Merge a LoRA update into a packed weight and re-quantize it.
+
+    Keras ``Dense`` (int4 diff), the merged-kernel helper: Step 1 dequantizes the kernel,
+    Step 2 adds ``(lora_alpha / lora_rank) * matmul(lora_kernel_a, lora_kernel_b)`` in the
+    float domain, Step 3 re-quantizes and packs. With the weight stored ``[N, K]`` the
+    update is ``delta[n, k] = c * sum_j b[n, j] * a[j, k]`` with ``b = lora_kernel_b^T``
+    ``[N, r]``, ``a = lora_kernel_a^T`` ``[r, K]`` and ``c = alpha / rank``.
+
+    Reading (fp32 throughout, each step rounded, in this order, so that the re-quantized
+    codes are a function of the inputs alone):
+      w      = fl32(q * s)                                   (the dequantized weight)
+      t      = 0;  for j = 0 .. r-1:  t = fl32(t + fl32(b[n, j] * a[j, k]))
+      w'     = fl32(w + fl32(c * t))
+    then :func:`quantize_rtn` on ``w'`` (this library's group-32 rule; Keras re-quantizes
+    into its own layouts). Returns ``(q', scales')`` as :func:`quantize_rtn`.
+    """
+    w = dequantize(codes, scales, K, "f32")
+    b = np.asarray(lora_b_t, dtype=np.float32)
+    a = np.asarray(lora_a_t, dtype=np.float32)
+    if b.shape[0] != w.shape[0] or a.shape[1] != K or b.shape[1] != a.shape[0]:
+        raise ValueError("lora_b_t must be [N, r] and lora_a_t [r, K]")
+    t = np.zeros_like(w, dtype=np.float32)
+    for j in range(b.shape[1]):
+        prod = (b[:, j:j + 1] * a[j:j + 1, :]).astype(np.float32)
+        t = (t + prod).astype(np.float32)
+    merged = (w + (np.float32(alpha_over_rank) * t).astype(np.float32)).astype(np.float32)
+    return quantize_rtn(merged)
+
+
+# ---------------------------------------------------------------------------
 # a6: asymmetric sub-channel variant with act-order g_idx
 # ---------------------------------------------------------------------------
 
