@@ -229,6 +229,28 @@ w4_status w4_expand_channel_scales(const float *scales, int64_t N, int64_t K, fl
                                    w4_stream_t stream);
 
 /*
+ * w4_lora_merge -- merge a LoRA update into a packed weight and re-quantize it.
+ * Keras page (keras/src/layers/core/dense.py, int4 diff), Dense's merged-kernel helper:
+ * dequantize the kernel, add (lora_alpha / lora_rank) * matmul(lora_kernel_a, lora_kernel_b)
+ * in the float domain, re-quantize, pack. With W stored [N, K]:
+ *     w  = fp32(value * scale)                        (as w4_dequantize, f32)
+ *     t  = 0; for j = 0 .. rank-1: t = fl32(t + fl32(lora_b_t[n][j] * lora_a_t[j][k]))
+ *     w' = fl32(w + fl32(alpha_over_rank * t))
+ * each step rounded in this order (no fused multiply-add), then the RTN rule of
+ * w4_quantize_rtn on w' -> codes_out, scales_out. Bit-identical to that definition.
+ *   lora_b_t  float32 [N, rank] (Keras lora_kernel_b transposed); lora_a_t float32 [rank, K]
+ *             (lora_kernel_a transposed); both may be NULL when rank == 0.
+ *   codes_out, scales_out  as w4_quantize_rtn's outputs; they may be codes and scales
+ *             themselves (in place).
+ *   d_status  as w4_quantize_rtn (a non-finite merged weight).
+ * Errors: W4_ERR_NULL, W4_ERR_SHAPE (sizes, rank < 0 or > 65536), W4_ERR_NONFINITE,
+ * W4_ERR_CUDA.
+ */
+w4_status w4_lora_merge(const uint8_t *codes, const float *scales, int64_t N, int64_t K, const float *lora_b_t,
+                        const float *lora_a_t, int64_t rank, float alpha_over_rank, uint8_t *codes_out,
+                        float *scales_out, int32_t *d_status, w4_stream_t stream);
+
+/*
  * w4_linear_backward_x -- input gradient of w4_linear: dx = dy . dequant(W).
  * Keras page (keras/src/layers/core/dense.py, int4 diff), _int4_call's grad_fn:
  * inputs_grad = matmul(upstream, transpose(float_kernel)); PaddleNLP page

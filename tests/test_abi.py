@@ -155,3 +155,13 @@ def test_channel_host_checks(w4):
     assert L.w4_quantize_rtn_channel(FAKE, 0, 64, FAKE, FAKE, None, None) == 2
     assert L.w4_expand_channel_scales(FAKE, 4, 0, FAKE, None) == 2
     assert L.w4_expand_channel_scales(None, 4, 64, FAKE, None) == 1
+
+
+def test_lora_host_checks(w4):
+    L = w4.lib
+    FAKE = ctypes.c_void_p(0x1000)
+    c = ctypes.c_float(1.0)
+    assert L.w4_lora_merge(None, FAKE, 4, 64, FAKE, FAKE, 2, c, FAKE, FAKE, None, None) == 1
+    assert L.w4_lora_merge(FAKE, FAKE, 4, 64, None, FAKE, 2, c, FAKE, FAKE, None, None) == 1
+    assert L.w4_lora_merge(FAKE, FAKE, 4, 64, FAKE, FAKE, -1, c, FAKE, FAKE, None, None) == 2
+    assert L.w4_lora_merge(FAKE, FAKE, 0, 64, FAKE, FAKE, 2, c, FAKE, FAKE, None, None) == 2

@@ -33,7 +33,7 @@ EXPORTS = (
     "w4_asym_prepare", "w4_linear_asym_gidx", "w4_linear_asym_gidx_noalloc", "w4_validate", "w4_validate_asym",
     "w4_set_weight_prefetch", "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
     "w4_dequantize_q4_0", "w4_linear_q4_0", "w4_linear_backward_x_workspace_bytes", "w4_linear_backward_x",
-    "w4_quantize_rtn_channel", "w4_expand_channel_scales",
+    "w4_quantize_rtn_channel", "w4_expand_channel_scales", "w4_lora_merge",
 )
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -60,6 +60,7 @@ _SIGS = {
     "w4_linear_backward_x": [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _i32, _vp, _sz, _vp],
     "w4_quantize_rtn_channel": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
     "w4_expand_channel_scales": [_vp, _i64, _i64, _vp, _vp],
+    "w4_lora_merge": [_vp, _vp, _i64, _i64, _vp, _vp, _i64, ctypes.c_float, _vp, _vp, _vp, _vp],
 }
 _lib = None
 
@@ -169,6 +170,26 @@ def quantize_rtn_channel(W: torch.Tensor, status: torch.Tensor | None = None):
     _check(_load().w4_quantize_rtn_channel(_ptr(W), N, K, _ptr(codes), _ptr(scales), _ptr(status), _stream()),
            "w4_quantize_rtn_channel")
     return codes, scales
+
+
+def lora_merge(codes: torch.Tensor, scales: torch.Tensor, K: int, lora_b_t: torch.Tensor | None,
+               lora_a_t: torch.Tensor | None, alpha_over_rank: float, out=None, status: torch.Tensor | None = None):
+    """Merge ``alpha_over_rank * lora_b_t [N, r] . lora_a_t [r, K]`` into the packed weight and
+    re-quantize; returns ``(codes', scales')`` (``out`` may be ``(codes, scales)``: in place)."""
+    _need_cuda(codes, scales, lora_b_t, lora_a_t, status)
+    N = codes.shape[0]
+    r = 0 if lora_b_t is None else lora_b_t.shape[1]
+    if r and (lora_b_t.dtype != torch.float32 or lora_a_t is None or lora_a_t.dtype != torch.float32 or
+              lora_b_t.shape != (N, r) or lora_a_t.shape != (r, K)):
+        raise ValueError("lora_b_t must be float32 [N, r] and lora_a_t float32 [r, K]")
+    if out is None:
+        out = (torch.empty_like(codes), torch.empty_like(scales))
+    co, so = out
+    _need_cuda(co, so)
+    _check(_load().w4_lora_merge(_ptr(codes), _ptr(scales), N, K, _ptr(lora_b_t), _ptr(lora_a_t), r,
+                                 float(alpha_over_rank), _ptr(co), _ptr(so), _ptr(status), _stream()),
+           "w4_lora_merge")
+    return co, so
 
 
 def expand_channel_scales(scales: torch.Tensor, K: int) -> torch.Tensor:

@@ -380,6 +380,33 @@ w4_status w4_expand_channel_scales(const float *scales, int64_t N, int64_t K, fl
   return e == cudaSuccess ? W4_OK : cuda_fail(e);
 }
 
+w4_status w4_lora_merge(const uint8_t *codes, const float *scales, int64_t N, int64_t K, const float *lora_b_t,
+                        const float *lora_a_t, int64_t rank, float alpha_over_rank, uint8_t *codes_out,
+                        float *scales_out, int32_t *d_status, w4_stream_t stream) {
+  if (!codes || !scales || !codes_out || !scales_out) return W4_ERR_NULL;
+  if (rank > 0 && (!lora_b_t || !lora_a_t)) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || rank < 0 || rank > 65536) return W4_ERR_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t *status = d_status;
+  if (!status) {
+    const w4_status st = symbol_ptr(&status, g_quant_status);
+    if (st != W4_OK) return st;
+    const cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  cudaError_t e = w4i::launch_lora_merge(codes, scales, lora_b_t, lora_a_t, N, K, rank, alpha_over_rank, codes_out,
+                                         scales_out, status, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!d_status) {
+    int32_t host = 0;
+    e = cudaMemcpyAsync(&host, status, sizeof(host), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (host != 0) return W4_ERR_NONFINITE;
+  }
+  return W4_OK;
+}
+
 int w4_set_weight_prefetch(int enable) {
   return g_weight_prefetch.exchange(enable != 0 ? 1 : 0);
 }

@@ -102,6 +102,12 @@ cudaError_t launch_quantize_rtn_channel(const float *W, int64_t N, int64_t K, ui
 cudaError_t launch_expand_channel_scales(const float *scales, int64_t N, int64_t K, float *out,
                                          cudaStream_t stream);
 
+// LoRA merge: codes/scales + alpha_over_rank * lora_b_t . lora_a_t, re-quantized (RTN
+// group-32) into codes_out/scales_out (which may be the inputs). status as quantize.
+cudaError_t launch_lora_merge(const uint8_t *codes, const float *scales, const float *lora_b_t,
+                              const float *lora_a_t, int64_t N, int64_t K, int64_t r, float alpha_over_rank,
+                              uint8_t *codes_out, float *scales_out, int32_t *status, cudaStream_t stream);
+
 // Validation flag bits (w4_validate reports them in the page's order).
 enum : uint32_t {
   FLAG_SCALE = 1u << 0,
