@@ -142,6 +142,54 @@ def oracle_sample(frac_rows=8):
     return run, nbytes, f"oracle linear (dequantize + fp64 matmul) at M=1 on 1/{frac_rows} of the rows of each decode shape"
 
 
+def oracle_detail_samples(frac_rows=8):
+    """Bounded oracle samples for the detail rows that have a host-side baseline: name ->
+    (callable, payload bytes per call, text). 1/frac_rows of the rows of each shape."""
+    import oracle as O
+    import oracle.q4_0 as Q
+    out = {}
+    q4 = []
+    for N, K in workloads.Q4_0_SHAPES:
+        c = workloads.q4_0_case(N + K, 1, N, K, bias=False)
+        q4.append((c["x"], c["blocks"][: N // frac_rows], K))
+
+    def run_q4():
+        for x, blocks, K in q4:
+            Q.linear(x, blocks, K)
+    out["q4_0_decode_M1_step"] = (run_q4, sum(Q.payload_bytes(N // frac_rows, K) for N, K in workloads.Q4_0_SHAPES),
+                                  f"oracle Q4_0 linear at M=1 on 1/{frac_rows} of the rows of each decode shape")
+    N, K = workloads.BATCHED_SHAPE
+    c = workloads.decode_case(N, K, M=1, config=3)
+    n = N // frac_rows
+    q, sc = O.quantize_rtn(c["W"][:n])
+    codes = O.pack_nibbles(q)
+    _, dy = workloads.draw_x(np.random.default_rng([3, 1]), 1, n)
+
+    def run_bwd():
+        O.linear_backward_x(dy, codes, sc, K)
+    out["backward_x_M1_14336x4096"] = (run_bwd, payload(n, K) + 2 * n + 2 * K,
+                                       f"oracle input gradient at M=1 on 1/{frac_rows} of the rows of (14336,4096)")
+    return out
+
+
+def time_oracle(run, nbytes, text, seconds=3.0):
+    """The oracle's throughput on one bounded sample (GB/s of the sample's payload)."""
+    try:
+        run()
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            run()
+            reps += 1
+            if time.perf_counter() - t0 > seconds:
+                break
+        dt = time.perf_counter() - t0
+        return {"value": reps * nbytes / dt / 1e9, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": text + f"; {reps} repetitions in {dt:.1f} s"}
+    except Exception as e:  # a failed baseline is reported, it does not stop the bench
+        return {"value": None, "unit": "GB/s", "kind": "oracle", "error": str(e)[:200]}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -377,6 +425,17 @@ def main():
         dt = time.perf_counter() - t0
         cpu = {"value": reps * nbytes / dt / 1e9, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": text + f"; {reps} repetitions in {dt:.1f} s on {os.cpu_count()} host CPUs"}
+        if detail is not None:
+            try:
+                samples = oracle_detail_samples()
+            except Exception as e:
+                samples = {}
+                for name in ("q4_0_decode_M1_step", "backward_x_M1_14336x4096"):
+                    if name in detail:
+                        detail[name]["cpu_baseline"] = {"value": None, "kind": "oracle", "error": str(e)[:200]}
+            for name, (run_d, nb_d, text_d) in samples.items():
+                if name in detail:
+                    detail[name]["cpu_baseline"] = time_oracle(run_d, nb_d, text_d)
 
     if world > 1:
         dist.barrier()

@@ -56,3 +56,15 @@ def test_reference_arm_other_ranks_exit_quietly():
                         "--steps", "1", "--warmup", "1"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_detail_oracle_baselines_run_on_cpu():
+    sys.path.insert(0, ROOT)
+    import bench
+    samples = bench.oracle_detail_samples(frac_rows=64)
+    assert set(samples) == {"q4_0_decode_M1_step", "backward_x_M1_14336x4096"}
+    for name, (run, nbytes, text) in samples.items():
+        r = bench.time_oracle(run, nbytes, text, seconds=0.2)
+        assert r["kind"] == "oracle" and r["value"] > 0 and nbytes > 0, name
+    bad = bench.time_oracle(lambda: 1 / 0, 1, "x", seconds=0.1)
+    assert bad["value"] is None and "error" in bad
