@@ -297,7 +297,8 @@ cudaError_t launch_linear_backward_x(const __nv_bfloat16 *dy, int64_t M, const u
                                      int64_t N, int64_t K, void *dx, int dx_dtype, void *workspace,
                                      size_t workspace_bytes, cudaStream_t stream) {
   const size_t need = linear_backward_x_workspace(M, N, K);
-  if (bwd_fast(codes, scales, K) && (need == 0 || (workspace != nullptr && workspace_bytes >= need))) {
+  const bool chunks_fit = (M + bwd_tm(M) - 1) / bwd_tm(M) <= 65535;  // grid z of the streaming kernel
+  if (bwd_fast(codes, scales, K) && chunks_fit && (need == 0 || (workspace != nullptr && workspace_bytes >= need))) {
     const int64_t splits = need == 0 ? 1 : bwd_splits(M, N, K);
     float *part = static_cast<float *>(workspace);
     if (bwd_wide(M, K) && reinterpret_cast<uintptr_t>(codes) % 16 == 0) {
