@@ -165,3 +165,18 @@ def test_lora_host_checks(w4):
     assert L.w4_lora_merge(FAKE, FAKE, 4, 64, None, FAKE, 2, c, FAKE, FAKE, None, None) == 1
     assert L.w4_lora_merge(FAKE, FAKE, 4, 64, FAKE, FAKE, -1, c, FAKE, FAKE, None, None) == 2
     assert L.w4_lora_merge(FAKE, FAKE, 0, 64, FAKE, FAKE, 2, c, FAKE, FAKE, None, None) == 2
+
+
+def test_new_bindings_validate_arguments(w4):
+    import torch
+    f32 = torch.zeros((4, 64), dtype=torch.float32)
+    with pytest.raises(ValueError):  # CPU tensors: no fallback
+        w4.quantize_rtn_channel(f32)
+    with pytest.raises(ValueError):
+        w4.expand_channel_scales(torch.zeros(4), 64)
+    with pytest.raises(ValueError):
+        w4.linear_backward_x(torch.zeros((1, 4), dtype=torch.bfloat16), torch.zeros((4, 32), dtype=torch.uint8),
+                             torch.zeros((4, 2), dtype=torch.float32), 64)
+    with pytest.raises(ValueError):
+        w4.lora_merge(torch.zeros((4, 32), dtype=torch.uint8), torch.zeros((4, 2)), 64, torch.zeros((4, 2)),
+                      torch.zeros((2, 64)), 1.0)
