@@ -156,5 +156,25 @@ def test_mutant_amax_over_padding(monkeypatch):
     _fails(P.pin_rtn_worked)
 
 
+def _check_linear_variant(any_=False, swap=False, strict=False, signed=False):
+    def check(y_gpu, y_ref, bound, rtol=4e-3, atol=1e-6):
+        y = np.asarray(y_gpu, np.float64)
+        err = (y - y_ref) if signed else np.abs(y - y_ref)
+        allow = (atol * bound + rtol) if swap else (rtol * bound + atol)
+        passed = (err < allow) if strict else (err <= allow)
+        worst = float(np.max(err / allow)) if err.size else 0.0
+        return bool(np.any(passed) if any_ else np.all(passed)), worst
+    return check
+
+
+@pytest.mark.parametrize("kind", ["any_", "swap", "strict", "signed"])
+def test_mutant_check_linear(monkeypatch, kind):
+    """An acceptance test that passes if any element passes, swaps the relative and
+    absolute terms, rejects an error equal to its allowance, or forgets the absolute
+    value each fails the acceptance pin."""
+    monkeypatch.setattr(O, "check_linear", _check_linear_variant(**{kind: True}))
+    _fails(P.pin_check_linear)
+
+
 def test_pins_pass_unmutated():
     P.pin_rtn_invariants(O, workloads.linear_case(1, 1, 8, 100)["W"])

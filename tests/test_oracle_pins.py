@@ -188,6 +188,34 @@ def pin_linear_worked(o):
     assert np.array_equal(bound[0], _floats(g["bound"])), bound
 
 
+def pin_check_linear(o):
+    """The acceptance rule ``|y - y_ref| <= 4e-3 * bound + 1e-6`` (the linear tolerance),
+    element by element, with values chosen so that every allowance is an exact double:
+    ``4e-3 * 1000`` rounds to exactly 4, so the allowance there is ``4 + 1e-6``; with a
+    zero bound it is ``1e-6``. An error equal to the allowance passes, the next double
+    above it fails, an error below ``y_ref`` counts as much as one above, and one bad
+    element (or a NaN) among many fails the whole output."""
+    y_ref = np.zeros((4, 2500))
+    bound = np.full((4, 2500), 1000.0)
+    bound[1] = 0.0
+    allow = np.where(bound > 0, 4.000001, 1e-6)
+    assert np.array_equal(4e-3 * bound + 1e-6, allow)
+    ok, worst = o.check_linear(y_ref + allow, y_ref, bound)
+    assert ok and worst == 1.0, (ok, worst)
+    ok, _ = o.check_linear(y_ref - allow, y_ref, bound)
+    assert ok
+    for m, n, sign in [(0, 7, 1.0), (1, 2499, -1.0), (3, 1234, 1.0)]:
+        y = y_ref + 0.5 * allow
+        y[m, n] = sign * np.nextafter(allow[m, n], np.inf)
+        ok, worst = o.check_linear(y, y_ref, bound)
+        assert not ok and worst > 1.0, (m, n, ok, worst)
+    y = y_ref.copy()
+    y[2, 5] = np.nan
+    assert not o.check_linear(y, y_ref, bound)[0]
+    ok, worst = o.check_linear(y_ref + 0.25 * allow, y_ref, bound)
+    assert ok and worst == 0.25
+
+
 def pin_linear_one_hot(o):
     """x = e_k picks column k of the dequantized weight (plus the bias)."""
     rng = np.random.default_rng(11)
@@ -345,6 +373,10 @@ def test_dequant_closed_form():
 
 def test_linear_worked_example():
     pin_linear_worked(O)
+
+
+def test_check_linear_acceptance():
+    pin_check_linear(O)
 
 
 def test_linear_one_hot():
