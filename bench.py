@@ -45,6 +45,36 @@ ROTATE = 4
 GRAPH_CHUNK = 1000  # steps per captured graph
 
 
+WARM_SECONDS = 0.3  # untimed load before the timed regions
+REGION_TARGET_S = 0.5  # total time of the repeated timed regions (at least MIN_REPEATS)
+MIN_REPEATS, MAX_REPEATS = 5, 51
+
+
+def repeats(steps, est_us_per_step=25.0):
+    """How many times the K-step timed region is repeated: enough regions to give a median
+    and p10/p90, about REGION_TARGET_S seconds in all."""
+    n = int(REGION_TARGET_S / max(steps * est_us_per_step * 1e-6, 1e-9))
+    return max(MIN_REPEATS, min(MAX_REPEATS, n))
+
+
+def spread(values):
+    """Median, p10 and p90 (linear interpolation) of a list of region times."""
+    v = np.sort(np.asarray(values, dtype=np.float64))
+    return {"median": float(np.median(v)), "p10": float(np.percentile(v, 10)),
+            "p90": float(np.percentile(v, 90)), "n": int(v.size)}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def payload(N, K):
     return N * ((K + 1) // 2) + 4 * N * ((K + 31) // 32)
 
@@ -325,21 +355,32 @@ def main():
 
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid)
-    time.sleep(0.2)
+    # untimed load until the clocks have settled (an idle GPU needs some time to ramp up)
+    t_w = time.perf_counter()
+    while time.perf_counter() - t_w < WARM_SECONDS:
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize()
+    # the K timed steps, R times over: each region is exactly the K steps, bracketed by a
+    # barrier and a synchronize on both sides; the line reports the median region
+    region_ms = []
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_start.record(stream)
-    for g in graphs:
-        g.replay()
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    for _ in range(repeats(args.steps)):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for g in graphs:
+            g.replay()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        region_ms.append(max_over_ranks(t_start.elapsed_time(t_end), dev))
     clocks = sampler.stop()
-    ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    dist_ms = spread(region_ms)
+    ms = dist_ms["median"]
 
     launches = args.steps * len(shapes)
     hbm_peak, tc_peak, tc_sus, peak_kind = peaks()
@@ -424,7 +465,24 @@ def main():
                 break
         dt = time.perf_counter() - t0
         cpu = {"value": reps * nbytes / dt / 1e9, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": text + f"; {reps} repetitions in {dt:.1f} s on {os.cpu_count()} host CPUs"}
+               "sample": text + f"; {reps} repetitions in {dt:.1f} s on {os.cpu_count()} host CPUs",
+               "cpu_model": cpu_model(), "host_cpus": os.cpu_count()}
+        try:  # the same sample on one thread
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                run()
+                t0 = time.perf_counter()
+                reps1 = 0
+                while True:
+                    run()
+                    reps1 += 1
+                    if time.perf_counter() - t0 > 5.0:
+                        break
+                dt1 = time.perf_counter() - t0
+            cpu["single_thread"] = {"value": reps1 * nbytes / dt1 / 1e9, "unit": UNIT, "cores": 1,
+                                    "sample": text + f"; {reps1} repetitions in {dt1:.1f} s"}
+        except Exception as e:
+            cpu["single_thread"] = {"value": None, "error": str(e)[:200]}
         if detail is not None:
             try:
                 samples = oracle_detail_samples()
@@ -453,10 +511,15 @@ def main():
         "config": {"workload": "decode GEMV M=1: (N,K) = (4096,4096), (14336,4096), (4096,14336); "
                                "RTN group-32 int4 + fp32 scales from W~N(0,0.02^2); x bf16 ~N(0,1); no bias",
                    "l2": f"inputs larger than L2: {ROTATE} rotating weight copies, {ROTATE * step_bytes / 2**20:.0f} MiB",
-                   "timing": "CUDA graphs of <=1000 steps replayed back to back, CUDA events on the launching stream around the replays",
+                   "timing": "CUDA graphs of <=1000 steps replayed back to back, CUDA events on the launching stream "
+                             f"around the replays; {WARM_SECONDS} s of untimed replays first; the K-step region "
+                             f"timed {dist_ms['n']} times (barrier + synchronize around each), value from the median",
                    "launch": "programmatic dependent launch; weights prefetched before the previous GEMV ends (weights constant)",
                    "parallelism": f"replicas x{world}"},
         "clocks": clocks,
+        "region_ms": {k: dist_ms[k] for k in ("median", "p10", "p90", "n")},
+        "value_p10_p90": [job_value(args.steps * step_bytes, world, dist_ms["p90"]),
+                          job_value(args.steps * step_bytes, world, dist_ms["p10"])],
         "gpu_launches": launches,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps,
@@ -520,7 +583,8 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
             fl = 2.0 * M * N * K
             return ([lambda c=c, s=s: w4.linear(x, c, s, K, bias=bias, out=y) for c, s in copies],
                     lambda us: {"us": us, "weight_gbs": payload(N, K) / us / 1e3,
-                                "frac_hbm": payload(N, K) / us / 1e3 / hbm_peak, "tflops": fl / us / 1e6})
+                                "frac_hbm": payload(N, K) / us / 1e3 / hbm_peak, "tflops": fl / us / 1e6,
+                                "frac_tensor": fl / us / 1e6 / tc_peak})
         return make
 
     def prefill(M, N, K):
@@ -552,7 +616,8 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
             return ([lambda c=c, s_=s_, z_=z_: w4.linear_asym_gidx(x, c, s_, z_, gi, perm=perm, bias=b, out=y,
                                                                    workspace=ws) for c, s_, z_ in copies],
                     lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak,
-                                "tflops": fl / us / 1e6})
+                                "tflops": fl / us / 1e6, "frac_tensor": fl / us / 1e6 / tc_peak,
+                                "bound": "hbm" if M <= 16 else "tensor"})
         return make
 
     def q4_0_decode():
