@@ -172,10 +172,12 @@ w4_status w4_linear_asym_gidx(const void *x, int64_t M, const uint8_t *codes,
  * workspace_bytes): the scratch memory lives in one fixed 16 MiB array inside the library,
  * present on every GPU that loads the library until the process exits.
  *   - The call allocates nothing (no cudaMalloc / cudaFree, no allocating library routine).
- *   - Shapes whose scratch (w4_linear_asym_workspace_bytes) exceeds 16 MiB -- M * K bf16
- *     activations, e.g. M = 2048 at K = 4096 -- return W4_ERR_SHAPE.
- *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress
- *     with that device current); make that first call before any stream capture.
+ *   - The limit is M * K * 2 bytes (the activations gathered in bf16) <= 16 MiB, whichever
+ *     kernel serves the shape: M = 2048 at K = 4096 is exactly 16 MiB and is accepted;
+ *     M = 2049 or M = 4096 at K = 4096 return W4_ERR_SHAPE.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress); the first call on a device also loads the library's device
+ *     code there, so make that first call before any stream capture.
  *   - All calls share the array and it keeps the last call's contents (each call overwrites
  *     what it reads, so nothing needs clearing). Calls that overlap on the GPU -- on
  *     different streams, or concurrently from several host threads -- race on it.
@@ -331,6 +333,16 @@ int w4_set_weight_prefetch(int enable);
  * synchronizes the device and clears it. */
 w4_status w4_device_error(void);
 
+/*
+ * w4_selftest_wait_timeout -- diagnostic with no counterpart on the source pages: launches one
+ * CTA on `stream` that waits, through the same bounded wait every kernel of the library uses,
+ * on a barrier nothing arrives on, with a limit of `limit_ns` nanoseconds (1 .. 1e9). The wait
+ * expires and records W4_ERR_TIMEOUT in the error word that w4_device_error() reads, exactly
+ * as an expired wait in a real kernel would; no copy or MMA is in flight and the CUDA context
+ * stays usable. Returns W4_ERR_SHAPE for a limit outside the range, else the launch status.
+ */
+w4_status w4_selftest_wait_timeout(uint64_t limit_ns, w4_stream_t stream);
+
 /* The cudaError_t of the last call that returned W4_ERR_CUDA (0 if none). */
 int w4_last_cuda_error(void);
 
@@ -339,6 +351,17 @@ const char *w4_status_string(w4_status status);
 
 /* Library ABI version (major * 100 + minor). */
 int w4_version(void);
+
+/*
+ * w4_last_linear_kernel -- name of the kernel family that the calling thread's last
+ * w4_linear / w4_linear_asym_gidx / w4_linear_asym_gidx_noalloc call launched: "gemv_tma",
+ * "gather_x+gemv_tma", "gemv_rows", "gemv_mma", "gemv", "gemm_tc", "gather_x+gemm_tc" or
+ * "linear_generic" ("none" before the first call on the thread). A static string owned by the
+ * library; set only when a call got as far as launching. For tests and profiling: the choice
+ * depends on M, the shape, the alignment of the arrays and the workspace (no counterpart on
+ * the source pages).
+ */
+const char *w4_last_linear_kernel(void);
 
 #ifdef __cplusplus
 }

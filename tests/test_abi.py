@@ -180,3 +180,10 @@ def test_new_bindings_validate_arguments(w4):
     with pytest.raises(ValueError):
         w4.lora_merge(torch.zeros((4, 32), dtype=torch.uint8), torch.zeros((4, 2)), 64, torch.zeros((4, 2)),
                       torch.zeros((2, 64)), 1.0)
+
+
+def test_wait_selftest_host_checks(w4):
+    """The wait self-test refuses a zero limit and one above the library's own 1 s limit
+    before anything is enqueued."""
+    assert w4.STATUS[w4.lib.w4_selftest_wait_timeout(0, None)] == "SHAPE"
+    assert w4.STATUS[w4.lib.w4_selftest_wait_timeout(10**9 + 1, None)] == "SHAPE"

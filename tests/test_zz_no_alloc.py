@@ -65,7 +65,38 @@ def test_noalloc_matches_workspace_entry_point_twice(w4):
 
 def test_noalloc_rejects_shapes_above_its_scratch(w4):
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check fails first
-    # 4096 x 4096 bf16 activations need 32 MiB of scratch, above the 16 MiB array
-    st = w4.lib.w4_linear_asym_gidx_noalloc(fake, 4096, fake, fake, fake, fake, fake, 256, 4096, 32, None, fake,
-                                            0, None)
-    assert w4.STATUS[st] == "SHAPE"
+    # 4096 x 4096 bf16 activations need 32 MiB of scratch, above the 16 MiB array; 2049 rows
+    # are the first row count above it at K = 4096; the limit holds whichever kernel would
+    # serve the shape (n_groups = 3 here keeps it off the tensor-core path)
+    for M, n_groups in [(4096, 32), (2049, 32), (2049, 3), (1 << 40, 32)]:
+        st = w4.lib.w4_linear_asym_gidx_noalloc(fake, M, fake, fake, fake, fake, fake, 256, 4096, n_groups, None,
+                                                fake, 0, None)
+        assert w4.STATUS[st] == "SHAPE", (M, n_groups)
+
+
+def test_noalloc_at_its_limit(w4):
+    """M = 2048 at K = 4096 (the act-order prefill shape, N = 11008, 32 groups of 128) needs
+    exactly the 16 MiB of the array: accepted, equal to the workspace entry point on every
+    output and to the oracle on sampled activation rows."""
+    a = workloads.asym_random_codes(2048)
+    M, N, K, G = a["M"], a["N"], a["K"], a["n_groups"]
+    assert M * K * 2 == 16 << 20
+    g_idx = _dev(a["g_idx"])
+    sorted_codes, perm = w4.asym_prepare(_dev(a["codes"]), g_idx, K, G)
+    ds, dz, db = _dev(a["scales"]), _dev(a["zeros"]), _dev(a["bias"])
+    xd = _dev(a["x_bits"].view(np.int16)).view(torch.bfloat16)
+    y_na = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    st = w4.lib.w4_linear_asym_gidx_noalloc(
+        w4._ptr(xd), M, w4._ptr(sorted_codes), w4._ptr(ds), w4._ptr(dz), w4._ptr(g_idx), w4._ptr(perm),
+        N, K, G, w4._ptr(db), w4._ptr(y_na), 0, w4._stream())
+    assert st == 0, w4.STATUS[st]
+    y_ws = w4.linear_asym_gidx(xd, sorted_codes, ds, dz, g_idx, perm=perm, bias=db)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(2048).choice(M, 24, replace=False)
+    yr, bound = O.linear_asym_gidx(a["x"][rows], a["codes"], a["scales"], a["zeros"], a["g_idx"], K, a["bias"])
+    na = y_na.float().cpu().numpy().astype(np.float64)
+    ws = y_ws.float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(na, ws), "the two entry points run the same kernels on the same inputs"
+    ok, worst = O.check_linear(na[rows], yr, bound)
+    assert ok, worst
+    assert w4.device_error() == "OK"

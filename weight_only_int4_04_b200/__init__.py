@@ -33,7 +33,8 @@ EXPORTS = (
     "w4_asym_prepare", "w4_linear_asym_gidx", "w4_linear_asym_gidx_noalloc", "w4_validate", "w4_validate_asym",
     "w4_set_weight_prefetch", "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
     "w4_dequantize_q4_0", "w4_linear_q4_0", "w4_linear_backward_x_workspace_bytes", "w4_linear_backward_x",
-    "w4_quantize_rtn_channel", "w4_expand_channel_scales", "w4_lora_merge",
+    "w4_quantize_rtn_channel", "w4_expand_channel_scales", "w4_lora_merge", "w4_selftest_wait_timeout",
+    "w4_last_linear_kernel",
 )
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -61,6 +62,8 @@ _SIGS = {
     "w4_quantize_rtn_channel": [_vp, _i64, _i64, _vp, _vp, _vp, _vp],
     "w4_expand_channel_scales": [_vp, _i64, _i64, _vp, _vp],
     "w4_lora_merge": [_vp, _vp, _i64, _i64, _vp, _vp, _i64, ctypes.c_float, _vp, _vp, _vp, _vp],
+    "w4_selftest_wait_timeout": [ctypes.c_uint64, _vp],
+    "w4_last_linear_kernel": [],
 }
 _lib = None
 
@@ -82,6 +85,7 @@ def _load():
         handle.w4_linear_asym_workspace_bytes.restype = ctypes.c_size_t
         handle.w4_linear_backward_x_workspace_bytes.restype = ctypes.c_size_t
         handle.w4_status_string.restype = ctypes.c_char_p
+        handle.w4_last_linear_kernel.restype = ctypes.c_char_p
         _lib = handle
     return _lib
 
@@ -445,3 +449,14 @@ def set_weight_prefetch(enable: bool) -> bool:
 
 def device_error() -> str:
     return STATUS[_load().w4_device_error()]
+
+
+def last_linear_kernel() -> str:
+    """Kernel family the calling thread's last linear call launched (``"none"`` before any)."""
+    return _load().w4_last_linear_kernel().decode()
+
+
+def selftest_wait_timeout(limit_ns: int) -> None:
+    """Make one bounded device wait expire after ``limit_ns`` (diagnostic; see the header):
+    the next ``device_error()`` reports ``"TIMEOUT"``."""
+    _check(_load().w4_selftest_wait_timeout(int(limit_ns), _stream()), "selftest_wait_timeout")

@@ -136,10 +136,12 @@ __global__ void __launch_bounds__(threads_for(BN), 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err)) break;
+        issued = kb + 1;
         mbar_arrive_expect_tx(&full_load[s], L::TX);
         tma_load_2d(smem + L::OFF_B + s * L::B_BYTES, &tmap_x, kb * BK, static_cast<int32_t>(m0), &full_load[s]);
         tma_load_2d(smem + L::OFF_C + s * C_BYTES, &tmap_codes, kb * (BK / 2), static_cast<int32_t>(n0),
@@ -153,6 +155,9 @@ __global__ void __launch_bounds__(threads_for(BN), 1)
           tma_load_2d(smem + L::OFF_Z + s * Z_BYTES, &tmap_zeros, gs & ~15, static_cast<int32_t>(n0), &full_load[s]);
         }
       }
+      // the copies issued land before the CTA may exit (see w4_sync.cuh, abort path)
+      for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
+        mbar_drain(&full_load[kb % STAGES], static_cast<uint32_t>(kb / STAGES) & 1u, err);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -173,6 +178,9 @@ __global__ void __launch_bounds__(threads_for(BN), 1)
         umma_commit(&empty[s]);
       }
       umma_commit(acc_full);
+      // every MMA issued has finished before the CTA frees its tensor memory (the epilogue
+      // stops waiting on an abort)
+      mbar_drain(acc_full, 0u, err);
     }
   } else {
     // ---- dequantize into the A stages ----

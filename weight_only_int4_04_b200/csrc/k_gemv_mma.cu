@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_mma_kernel(const LinearParam
   if (warp == kConsumerWarps) {
     // ---- producer: per row one bulk copy per array into the padded slot layout ----
     if (lane == 0) {
+      int issued = 0;
       for (int s = 0; s < nstages; ++s) {
         // stage s belongs to warp group s % ngroups, which walks its own ring of spg slots
         const int kq = s / g.ngroups;
@@ -154,6 +155,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_mma_kernel(const LinearParam
           if (ASYM)
             bulk_copy_g2s(base + g.zeros_off + r * g.zero_pitch, p.zeros + (r0 + r) * g.SG, zb, &full[slot]);
         }
+        issued = s + 1;
+      }
+      // the copies issued land before the CTA may exit (see w4_sync.cuh, abort path); each
+      // slot's latest phase lies in the last ngroups * spg stages, one stage per slot
+      const int ring = g.ngroups * g.spg;
+      for (int s = issued - ring < 0 ? 0 : issued - ring; s < issued; ++s) {
+        const int kq = s / g.ngroups;
+        mbar_drain(&full[(s % g.ngroups) * g.spg + kq % g.spg], static_cast<uint32_t>(kq / g.spg) & 1u, err);
       }
     }
     return;

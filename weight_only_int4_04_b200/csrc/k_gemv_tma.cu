@@ -227,8 +227,11 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
       int32_t row = static_cast<int32_t>(rb_begin * kRowsPerBlock);
       // weights first when they may be prefetched (they do not depend on the previous kernel)
       const int early = p.prefetch ? (total < p.S ? total : p.S) : 0;
+      int issued = 0;        // stages whose copies were issued
+      bool x_issued = false;  // the activation copies (several rows)
       for (int i = 0; i <= total; ++i) {
         if (NT != 0 && (!ASYM || p.x_sorted) && i == early) {
+          x_issued = true;
           // x is written by the previous kernel: copy it only once that kernel has finished.
           // (M = 1: the consumers load it themselves, in one round trip.)
           grid_dependency_wait();
@@ -272,6 +275,7 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
             tma_load_2d_hint(st + W * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
                         &full[slot], pol);
         }
+        issued = i + 1;
         if (++kc == p.SPR) {
           kc = 0;
           row += kRowsPerBlock;
@@ -281,6 +285,11 @@ __global__ void __launch_bounds__(32 * (warps_for(NT) + 1), NT == 0 ? 2 : 1)
           phase ^= 1u;
         }
       }
+      // every copy issued must land before the CTA may exit (the consumers stop waiting on
+      // an abort): the last S stages hold distinct slots, each at its latest phase
+      for (int i = issued - p.S < 0 ? 0 : issued - p.S; i < issued; ++i)
+        mbar_drain(&full[i % p.S], static_cast<uint32_t>(i / p.S) & 1u, err);
+      if (x_issued) mbar_drain(x_full, 0u, err);
     }
     return;
   }

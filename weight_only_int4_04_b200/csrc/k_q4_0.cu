@@ -115,11 +115,13 @@ __global__ void __launch_bounds__(32 * (kQWarps + 1), 2)
       uint32_t phase = 0;
       int32_t row = static_cast<int32_t>(rb_begin * kQRows);
       if (!p.prefetch) grid_dependency_wait();  // the blocks may come from the previous kernel
+      int issued = 0;
       for (int i = 0; i < total; ++i) {
         if (!mbar_wait(&empty[slot], phase ^ 1u, abort_flag, err)) break;
         // whole-stage box; k-tiles past the row end read as zeros (and count as bytes)
         mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(kQStageBytes));
         tma_load_3d_hint(smem + slot * kQStageBytes, &tm_blocks, 0, row, kc * kQWarps, &full[slot], pol);
+        issued = i + 1;
         if (++kc == p.SPR) {
           kc = 0;
           row += kQRows;
@@ -129,6 +131,9 @@ __global__ void __launch_bounds__(32 * (kQWarps + 1), 2)
           phase ^= 1u;
         }
       }
+      // the copies issued land before the CTA may exit (see w4_sync.cuh, abort path)
+      for (int i = issued - kQStages < 0 ? 0 : issued - kQStages; i < issued; ++i)
+        mbar_drain(&full[i % kQStages], static_cast<uint32_t>(i / kQStages) & 1u, err);
     }
     return;
   }

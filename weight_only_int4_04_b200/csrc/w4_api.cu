@@ -7,9 +7,21 @@
 #include <cstring>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "w4_internal.cuh"
+#include "w4_sync.cuh"
 
 namespace {
+
+// NVTX range around each entry point (a push/pop pair: near-free unless a profiler is
+// attached, which then shows every call of the library on its timeline by name).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 thread_local int g_last_cuda_error = 0;
 
@@ -43,6 +55,9 @@ w4_status symbol_ptr(T **out, const T &sym) {
 // previous kernel of the stream has finished.
 std::atomic<int> g_weight_prefetch{0};
 
+// Kernel family the calling thread's last linear call launched (w4_last_linear_kernel).
+thread_local const char *t_last_kernel = "none";
+
 // Tensor-core GEMM is used above this M (and whenever the decode kernels do not apply).
 constexpr int64_t kTcMinM = 17;
 
@@ -60,15 +75,7 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
   // 128, activations that fit in shared memory), else for M = 1 the register-streaming GEMV
   // and for M <= 16 the bulk-copy mma.sync kernel; larger M -> the tcgen05 GEMM; the other
   // kernels take the shapes the fast paths cannot (unaligned rows, odd widths, unsorted
-  // act-order maps). W4_GEMV=rows|stream|mma picks an alternative small-M kernel (for
-  // comparisons only).
-  static const int m1_kernel = [] {
-    const char *v = getenv("W4_GEMV");
-    if (v != nullptr && strcmp(v, "stream") == 0) return 1;
-    if (v != nullptr && strcmp(v, "mma") == 0) return 2;
-    if (v != nullptr && strcmp(v, "rows") == 0) return 3;
-    return 0;
-  }();
+  // act-order maps). The kernel chosen is recorded for w4_last_linear_kernel().
   cudaError_t e;
   // act-order beyond one short row: x is gathered into sorted column order once per call,
   // into the workspace, so that no CTA of the GEMV has to gather it (one row: every CTA
@@ -76,7 +83,7 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
   const bool asym_gather = p.asym && !w4i::gemv_tma_gathers_x(p);
   const bool ws_gather = workspace != nullptr && workspace_bytes >= w4i::gemm_tc_asym_workspace(p.M, p.K) &&
                          p.K % 8 == 0;
-  if (m1_kernel == 0 && w4i::gemv_tma_supports(p) && (!asym_gather || ws_gather)) {
+  if (w4i::gemv_tma_supports(p) && (!asym_gather || ws_gather)) {
     const __nv_bfloat16 *xs = nullptr;
     e = cudaSuccess;
     if (asym_gather) {
@@ -85,19 +92,23 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
     }
     if (e == cudaSuccess)
       e = w4i::launch_gemv_tma(p, g_weight_prefetch.load(std::memory_order_relaxed) != 0, xs, err, stream);
-  } else if ((m1_kernel == 0 || m1_kernel == 3) && w4i::gemv_rows_supports(p)) {
+    t_last_kernel = asym_gather ? "gather_x+gemv_tma" : "gemv_tma";
+  } else if (w4i::gemv_rows_supports(p)) {
     e = w4i::launch_gemv_rows(p, stream);
-  } else if (m1_kernel != 2 && w4i::gemv_stream_supports(p)) {
-    e = w4i::launch_gemv_stream(p, err, stream);
+    t_last_kernel = "gemv_rows";
   } else if (w4i::gemv_mma_supports(p)) {
     e = w4i::launch_gemv_mma(p, err, stream);
+    t_last_kernel = "gemv_mma";
   } else if (w4i::gemv_supports(p)) {
     e = w4i::launch_gemv(p, stream);
+    t_last_kernel = "gemv";
   } else if (p.M > 4 && w4i::gemm_tc_supports(p) &&
              (!p.asym || (workspace != nullptr && workspace_bytes >= w4i::gemm_tc_asym_workspace(p.M, p.K)))) {
     e = w4i::launch_gemm_tc(p, err, stream, workspace);
+    t_last_kernel = p.asym ? "gather_x+gemm_tc" : "gemm_tc";
   } else {
     e = w4i::launch_linear_generic(p, stream);
+    t_last_kernel = "linear_generic";
   }
   return e == cudaSuccess ? W4_OK : cuda_fail(e);
 }
@@ -107,6 +118,8 @@ w4_status run_linear(const w4i::LinearParams &p, void *workspace, size_t workspa
 extern "C" {
 
 int w4_version(void) { return 100; }
+
+const char *w4_last_linear_kernel(void) { return t_last_kernel; }
 
 int w4_last_cuda_error(void) { return g_last_cuda_error; }
 
@@ -133,6 +146,7 @@ const char *w4_status_string(w4_status s) {
 
 w4_status w4_quantize_rtn(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
                           int32_t *d_status, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_quantize_rtn");
   if (!W || !codes || !scales) return W4_ERR_NULL;
   if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -157,6 +171,7 @@ w4_status w4_quantize_rtn(const float *W, int64_t N, int64_t K, uint8_t *codes, 
 
 w4_status w4_dequantize(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
                         int format_version, w4_dtype out_dtype, void *out, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_dequantize");
   if (!codes || !scales || !out) return W4_ERR_NULL;
   if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
   if (format_version != 1 && format_version != 2) return W4_ERR_VERSION;
@@ -177,6 +192,7 @@ size_t w4_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 w4_status w4_linear(const void *x, int64_t M, const uint8_t *codes, const float *scales, int64_t N,
                     int64_t K, const float *bias, void *y, w4_dtype y_dtype, void *workspace,
                     size_t workspace_bytes, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_linear");
   if (!x || !codes || !scales || !y) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || M < 1 || M > kMaxRows) return W4_ERR_SHAPE;
   if (y_dtype != W4_BF16 && y_dtype != W4_F32) return W4_ERR_DTYPE;
@@ -207,6 +223,7 @@ size_t w4_linear_asym_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t n
 
 w4_status w4_asym_prepare(const uint8_t *codes_in, const int32_t *g_idx, int64_t N, int64_t K,
                           int64_t n_groups, uint8_t *codes_out, int32_t *perm, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_asym_prepare");
   if (!codes_in || !g_idx || !codes_out || !perm) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || n_groups < 1 || n_groups > K) return W4_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -231,6 +248,7 @@ w4_status w4_linear_asym_gidx(const void *x, int64_t M, const uint8_t *codes, co
                               int64_t N, int64_t K, int64_t n_groups, const float *bias, void *y,
                               w4_dtype y_dtype, void *workspace, size_t workspace_bytes,
                               w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_linear_asym_gidx");
   if (!x || !codes || !scales || !zeros || !g_idx || !y) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || M < 1 || M > kMaxRows || n_groups < 1 || n_groups > K) return W4_ERR_SHAPE;
   if (y_dtype != W4_BF16 && y_dtype != W4_F32) return W4_ERR_DTYPE;
@@ -274,6 +292,7 @@ static w4_status run_validate(const uint8_t *codes, const float *scales, const i
 
 w4_status w4_validate(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
                       int format_version, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_validate");
   if (!codes || !scales) return W4_ERR_NULL;
   if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
   if (format_version != 1 && format_version != 2) return W4_ERR_VERSION;
@@ -290,6 +309,7 @@ w4_status w4_validate(const uint8_t *codes, const float *scales, int64_t N, int6
 w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8_t *zeros,
                            const int32_t *g_idx, int64_t N, int64_t K, int64_t n_groups,
                            w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_validate_asym");
   if (!codes || !scales || !zeros || !g_idx) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || n_groups < 1 || n_groups > K) return W4_ERR_SHAPE;
   uint32_t f = 0;
@@ -305,6 +325,7 @@ w4_status w4_validate_asym(const uint8_t *codes, const float *scales, const int8
 
 w4_status w4_dequantize_q4_0(const uint8_t *blocks, int64_t N, int64_t K, w4_dtype out_dtype, void *out,
                              w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_dequantize_q4_0");
   if (!blocks || !out) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || K % 32 != 0) return W4_ERR_SHAPE;
   if (out_dtype != W4_BF16 && out_dtype != W4_F16 && out_dtype != W4_F32 && out_dtype != W4_F64)
@@ -316,6 +337,7 @@ w4_status w4_dequantize_q4_0(const uint8_t *blocks, int64_t N, int64_t K, w4_dty
 
 w4_status w4_linear_q4_0(const void *x, int64_t M, const uint8_t *blocks, int64_t N, int64_t K,
                          const float *bias, void *y, w4_dtype y_dtype, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_linear_q4_0");
   if (!x || !blocks || !y) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || K % 32 != 0 || M < 1 || M > kMaxRows) return W4_ERR_SHAPE;
   if (y_dtype != W4_BF16 && y_dtype != W4_F32) return W4_ERR_DTYPE;
@@ -335,6 +357,7 @@ size_t w4_linear_backward_x_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 w4_status w4_linear_backward_x(const void *dy, int64_t M, const uint8_t *codes, const float *scales, int64_t N,
                                int64_t K, void *dx, w4_dtype dx_dtype, void *workspace, size_t workspace_bytes,
                                w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_linear_backward_x");
   if (!dy || !codes || !scales || !dx) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || M < 1 || M > kMaxRows) return W4_ERR_SHAPE;
   if (dx_dtype != W4_BF16 && dx_dtype != W4_F32) return W4_ERR_DTYPE;
@@ -349,6 +372,7 @@ w4_status w4_linear_backward_x(const void *dy, int64_t M, const uint8_t *codes, 
 
 w4_status w4_quantize_rtn_channel(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
                                   int32_t *d_status, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_quantize_rtn_channel");
   if (!W || !codes || !scales) return W4_ERR_NULL;
   if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -373,6 +397,7 @@ w4_status w4_quantize_rtn_channel(const float *W, int64_t N, int64_t K, uint8_t 
 
 w4_status w4_expand_channel_scales(const float *scales, int64_t N, int64_t K, float *scales_out,
                                    w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_expand_channel_scales");
   if (!scales || !scales_out) return W4_ERR_NULL;
   if (!sizes_ok(N, K)) return W4_ERR_SHAPE;
   const cudaError_t e =
@@ -383,6 +408,7 @@ w4_status w4_expand_channel_scales(const float *scales, int64_t N, int64_t K, fl
 w4_status w4_lora_merge(const uint8_t *codes, const float *scales, int64_t N, int64_t K, const float *lora_b_t,
                         const float *lora_a_t, int64_t rank, float alpha_over_rank, uint8_t *codes_out,
                         float *scales_out, int32_t *d_status, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_lora_merge");
   if (!codes || !scales || !codes_out || !scales_out) return W4_ERR_NULL;
   if (rank > 0 && (!lora_b_t || !lora_a_t)) return W4_ERR_NULL;
   if (!sizes_ok(N, K) || rank < 0 || rank > 65536) return W4_ERR_SHAPE;
@@ -409,6 +435,15 @@ w4_status w4_lora_merge(const uint8_t *codes, const float *scales, int64_t N, in
 
 int w4_set_weight_prefetch(int enable) {
   return g_weight_prefetch.exchange(enable != 0 ? 1 : 0);
+}
+
+w4_status w4_selftest_wait_timeout(uint64_t limit_ns, w4_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > w4i::kWaitLimitNs) return W4_ERR_SHAPE;
+  int32_t *err = nullptr;
+  const w4_status st = symbol_ptr(&err, g_device_error);
+  if (st != W4_OK) return st;
+  const cudaError_t e = w4i::launch_wait_selftest(limit_ns, err, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
 }
 
 w4_status w4_device_error(void) {

@@ -45,10 +45,6 @@ cudaError_t launch_linear_generic(const LinearParams &p, cudaStream_t stream);
 // fit this kernel (the caller then picks another).
 cudaError_t launch_gemv(const LinearParams &p, cudaStream_t stream);
 bool gemv_supports(const LinearParams &p);
-// Streaming decode GEMV (bulk-copy ring, one CTA per SM) for M = 1 and aligned rows.
-// `err` is the library's device error word (bounded waits report W4_ERR_TIMEOUT there).
-cudaError_t launch_gemv_stream(const LinearParams &p, int32_t *err, cudaStream_t stream);
-bool gemv_stream_supports(const LinearParams &p);
 // Register-streaming decode GEMV (M = 1): every lane prefetches its own code rows.
 cudaError_t launch_gemv_rows(const LinearParams &p, cudaStream_t stream);
 bool gemv_rows_supports(const LinearParams &p);
@@ -107,6 +103,11 @@ cudaError_t launch_expand_channel_scales(const float *scales, int64_t N, int64_t
 cudaError_t launch_lora_merge(const uint8_t *codes, const float *scales, const float *lora_b_t,
                               const float *lora_a_t, int64_t N, int64_t K, int64_t r, float alpha_over_rank,
                               uint8_t *codes_out, float *scales_out, int32_t *status, cudaStream_t stream);
+
+// Diagnostic: one CTA waits, with the library's bounded wait and a limit of limit_ns, on a
+// barrier that nothing arrives on, so the wait expires and records W4_ERR_TIMEOUT in `err`.
+// No copy or MMA is in flight; the kernel returns normally.
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t *err, cudaStream_t stream);
 
 // Validation flag bits (w4_validate reports them in the page's order).
 enum : uint32_t {

@@ -3,6 +3,12 @@
 // sets a CTA-wide abort flag so that the remaining waits of the CTA give up at once; the
 // kernel then runs to its end on whatever data it has, and the host sees the error through
 // w4_device_error(). No wait can hang the GPU.
+//
+// Abort path: a CTA must not exit while bulk copies it issued can still write its shared
+// memory, nor free tensor memory that an MMA it issued may still write. So the thread that
+// issues the copies of a ring waits, before it returns, for every stage it issued to land
+// (mbar_drain: bounded, but deaf to the abort flag), and the MMA issuer waits for its last
+// commit before the CTA frees its tensor memory.
 #pragma once
 
 #include <stdint.h>
@@ -71,19 +77,36 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 // (timeout here or an abort raised elsewhere in the CTA). A caller must never wait for a
 // phase more than one ahead of the barrier's last completed phase (parity would alias).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          int32_t *err) {
+                                          int32_t *err, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 0;; ++n) {
     // The hint lets the hardware suspend the thread until the phase completes (it wakes on
     // completion, not on a timer), so a waiter takes no issue slots and resumes at once.
-    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    const uint32_t hint = limit_ns < 1000000u ? static_cast<uint32_t>(limit_ns) + 1u : 1000000u;
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
     if (n >= 32) __nanosleep(256);  // only if the suspend keeps returning early
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       if (err) atomicExch(err, static_cast<int32_t>(W4_ERR_TIMEOUT));
       return false;
+    }
+  }
+}
+
+// Wait for a phase that copies or MMAs this thread issued will complete, whatever the abort
+// flag says (their writes must land before the CTA exits or frees tensor memory). Bounded by
+// kWaitLimitNs like every other wait; gives up with W4_ERR_TIMEOUT recorded.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, int32_t *err) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t n = 0;; ++n) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return;
+    if (n >= 32) __nanosleep(256);
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (err) atomicExch(err, static_cast<int32_t>(W4_ERR_TIMEOUT));
+      return;
     }
   }
 }
