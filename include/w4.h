@@ -81,9 +81,12 @@ typedef enum { W4_BF16 = 0, W4_F16 = 1, W4_F32 = 2, W4_F64 = 3 } w4_dtype;
  *   codes    out, uint8 [N, ceil(K/2)];  scales  out, float32 [N, ceil(K/32)].
  *   d_status optional device int32: set to W4_ERR_NONFINITE if W holds NaN/Inf, left
  *            unchanged otherwise (the caller zeroes it). If NULL, the call synchronizes
- *            `stream` and returns W4_ERR_NONFINITE itself. Outputs are unspecified for a
- *            non-finite W. The results are bit-identical to the definition above (IEEE
- *            divide, no flush-to-zero).
+ *            `stream` and returns W4_ERR_NONFINITE itself, using one status word inside the
+ *            library that every NULL-d_status call (this one, w4_quantize_rtn_channel,
+ *            w4_lora_merge) shares: such calls must not overlap on the GPU (from several
+ *            host threads or streams at once) -- pass d_status when they may. Outputs are
+ *            unspecified for a non-finite W. The results are bit-identical to the
+ *            definition above (IEEE divide, no flush-to-zero).
  */
 w4_status w4_quantize_rtn(const float *W, int64_t N, int64_t K, uint8_t *codes, float *scales,
                           int32_t *d_status, w4_stream_t stream);
@@ -192,7 +195,8 @@ w4_status w4_linear_asym_gidx_noalloc(const void *x, int64_t M, const uint8_t *c
  * w4_validate -- the LoopQ content checks (page "loopq/packed_weight.py", validate) on a
  * device-resident packed weight, reported in the page's order: W4_ERR_VERSION (format not
  * 1 or 2), W4_ERR_SCALE, W4_ERR_HIGH_NIBBLE, W4_ERR_RESERVED_CODE (v1 only). Shape and
- * dtype are the caller's contract. Synchronizes `stream`.
+ * dtype are the caller's contract. Synchronizes `stream`. The flags live in one word inside
+ * the library shared by w4_validate and w4_validate_asym: calls must not overlap on the GPU.
  */
 w4_status w4_validate(const uint8_t *codes, const float *scales, int64_t N, int64_t K,
                       int format_version, w4_stream_t stream);

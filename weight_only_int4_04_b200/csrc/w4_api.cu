@@ -26,7 +26,9 @@ struct NvtxRange {
 thread_local int g_last_cuda_error = 0;
 
 // Device words: validation flags and the non-finite flag of a quantize call that was given
-// no status pointer. Calls that use them synchronize, so they are never shared in flight.
+// no status pointer. Calls that use them synchronize their stream before returning, so one
+// host thread never shares them in flight; calls from several threads or streams at once
+// would (the header tells callers to pass their own status word then).
 __device__ uint32_t g_validate_flags;
 __device__ int32_t g_quant_status;
 // Written by bounded device-side waits when they give up (read by w4_device_error).
