@@ -34,6 +34,7 @@ def _x(bits):
 SYM_CASES = [
     # (M, N, K, x_offset_bytes, expected kernel, why)
     (1, 300, 4096, 0, "gemv_tma", "M = 1, K a multiple of 128, aligned arrays"),
+    (1, 300, 2176, 0, "gemv_tma", "M = 1, K a multiple of 128 but not of 1024 (one 2-D box per k-tile)"),
     (8, 300, 2048, 0, "gemv_tma", "2 <= M <= 8: one n-tile"),
     (16, 300, 2048, 0, "gemv_tma", "9 <= M <= 16: two n-tiles"),
     (1, 300, 1056, 0, "gemv_rows", "M = 1, K % 128 != 0 (no TMA boxes), packed rows a multiple of 16 bytes"),
