@@ -638,6 +638,25 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
         return ([lambda r=r: step(r) for r in range(ROTATE)],
                 lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
 
+    def channel_decode():
+        # the headline's decode step on per-channel weights (one fp32 scale per row, read by
+        # the decode kernel: 0.5 bytes per weight + 4 per row)
+        sets, xs, ys, nb = [], [], [], 0
+        for N, K in workloads.DECODE_SHAPES:
+            c = workloads.decode_case(N, K)
+            codes, scales = w4.quantize_rtn_channel(torch.from_numpy(c["W"]).to(dev))
+            sets.append([(codes.clone(), scales.clone()) for _ in range(ROTATE)])
+            xs.append(bf16(c["x_bits"]))
+            ys.append(torch.empty((1, N), dtype=torch.bfloat16, device=dev))
+            nb += N * ((K + 1) // 2) + 4 * N
+
+        def step(r):
+            for j, (N, K) in enumerate(workloads.DECODE_SHAPES):
+                cd, sc = sets[j][r]
+                w4.linear_channel(xs[j], cd, sc, K, out=ys[j])
+        return ([lambda r=r: step(r) for r in range(ROTATE)],
+                lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
+
     def backward_x(M):
         # input gradient dx = dy . dequant(W) of the (14336, 4096) projection
         def make():
@@ -656,6 +675,7 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
         return make
 
     w = {"dequant_4096x4095_bf16": dequant_odd, "quantize_14336x4096": quantize, "q4_0_decode_M1_step": q4_0_decode,
+         "channel_decode_M1_step": channel_decode,
          "backward_x_M1_14336x4096": backward_x(1), "backward_x_M16_14336x4096": backward_x(16)}
     for M in workloads.BATCHED_M:
         w[f"batched_M{M}_14336x4096"] = batched(M)

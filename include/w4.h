@@ -235,6 +235,24 @@ w4_status w4_expand_channel_scales(const float *scales, int64_t N, int64_t K, fl
                                    w4_stream_t stream);
 
 /*
+ * w4_linear_channel -- the linear y = x . dequant(W)^T + bias for a per-channel weight: codes
+ * as w4_linear, scales float32 [N] (one per row). The dequantized weight is q * s[n]; the
+ * result agrees with w4_linear on the expanded scales within the linear tolerance (here the
+ * row's sum of code * x is scaled once instead of each group's).
+ *   M <= 16, K a multiple of 128, 16-byte aligned x and codes: a decode kernel that streams
+ *   the codes and one scale per row (0.5 bytes per weight instead of 0.625 with expanded
+ *   scales), no workspace.
+ *   Other calls: the scales are expanded into `workspace` (w4_linear_channel_workspace_bytes:
+ *   N * ceil(K/32) floats, 256-byte aligned) and the group-32 linear runs; W4_ERR_WORKSPACE if
+ *   it is missing or too small.
+ * Errors: W4_ERR_NULL, W4_ERR_SHAPE, W4_ERR_DTYPE (y bf16 or f32), W4_ERR_WORKSPACE, W4_ERR_CUDA.
+ */
+size_t w4_linear_channel_workspace_bytes(int64_t M, int64_t N, int64_t K);
+w4_status w4_linear_channel(const void *x, int64_t M, const uint8_t *codes, const float *scales, int64_t N,
+                            int64_t K, const float *bias, void *y, w4_dtype y_dtype, void *workspace,
+                            size_t workspace_bytes, w4_stream_t stream);
+
+/*
  * w4_lora_merge -- merge a LoRA update into a packed weight and re-quantize it.
  * Keras page (keras/src/layers/core/dense.py, int4 diff), Dense's merged-kernel helper:
  * dequantize the kernel, add (lora_alpha / lora_rank) * matmul(lora_kernel_a, lora_kernel_b)
@@ -360,7 +378,8 @@ int w4_version(void);
  * w4_last_linear_kernel -- name of the kernel family that the calling thread's last
  * w4_linear / w4_linear_asym_gidx / w4_linear_asym_gidx_noalloc call launched: "gemv_tma",
  * "gather_x+gemv_tma", "gemv_rows", "gemv_mma", "gemv", "gemm_tc", "gather_x+gemm_tc" or
- * "linear_generic" ("none" before the first call on the thread). A static string owned by the
+ * "linear_generic"; w4_linear_channel reports "gemv_tma_channel" or, after expanding the
+ * scales, the group-32 kernel it ran ("none" before the first call on the thread). A static string owned by the
  * library; set only when a call got as far as launching. For tests and profiling: the choice
  * depends on M, the shape, the alignment of the arrays and the workspace (no counterpart on
  * the source pages).

@@ -187,3 +187,12 @@ def test_wait_selftest_host_checks(w4):
     before anything is enqueued."""
     assert w4.STATUS[w4.lib.w4_selftest_wait_timeout(0, None)] == "SHAPE"
     assert w4.STATUS[w4.lib.w4_selftest_wait_timeout(10**9 + 1, None)] == "SHAPE"
+
+
+def test_linear_channel_host_checks(w4):
+    L = w4.lib
+    assert w4.STATUS[L.w4_linear_channel(None, 1, FAKE, FAKE, 4, 128, None, FAKE, 0, None, 0, None)] == "NULL"
+    assert w4.STATUS[L.w4_linear_channel(FAKE, 0, FAKE, FAKE, 4, 128, None, FAKE, 0, None, 0, None)] == "SHAPE"
+    assert w4.STATUS[L.w4_linear_channel(FAKE, 1, FAKE, FAKE, 4, 128, None, FAKE, 3, None, 0, None)] == "DTYPE"
+    assert int(L.w4_linear_channel_workspace_bytes(1, 64, 4096)) == 0
+    assert int(L.w4_linear_channel_workspace_bytes(17, 64, 4096)) == 64 * 128 * 4

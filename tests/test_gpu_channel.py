@@ -81,3 +81,69 @@ def test_channel_linear_and_gradient(w4, MNK):
     dxr, dbound = O.linear_backward_x(dy, rc, rs, K)
     ok, worst = O.check_linear(dx.cpu().numpy(), dxr, dbound)
     assert ok, (MNK, "dx", worst)
+
+
+# ---------------------------------------------------------------------------
+# w4_linear_channel: one scale per row read by the decode kernel (M <= 16), or expanded into
+# the workspace for the group-32 kernels (other shapes)
+# ---------------------------------------------------------------------------
+
+CHANNEL_LINEAR = [
+    # (M, N, K, kernel expected)
+    (1, 300, 4096, "gemv_tma_channel"),    # whole-stage 3-D boxes of codes
+    (1, 4100, 2176, "gemv_tma_channel"),   # K % 1024 != 0: 2-D boxes per k-tile, ragged rows
+    (1, 64, 14336, "gemv_tma_channel"),    # long rows: several stages per row block
+    (5, 300, 4096, "gemv_tma_channel"),    # one n-tile of activation rows
+    (16, 333, 2048, "gemv_tma_channel"),   # two n-tiles
+    (17, 300, 4096, "gemm_tc"),            # expanded scales, tensor-core GEMM
+    (3, 300, 1056, "gemv"),                # K % 128 != 0: expanded scales, CUDA-core GEMV
+    (1, 257, 1001, "linear_generic"),      # odd K
+]
+
+
+@pytest.mark.parametrize("case", CHANNEL_LINEAR, ids=[f"M{c[0]}-N{c[1]}-K{c[2]}" for c in CHANNEL_LINEAR])
+def test_linear_channel_matches_oracle(w4, case):
+    M, N, K, expect = case
+    c = workloads.linear_case(M * 5 + N + K, M, N, K, outliers=True)
+    q, s = O.quantize_rtn_channel(c["W"])
+    codes = O.pack_nibbles(q)
+    y = w4.linear_channel(bf16_dev(c["x_bits"]), dev(codes), dev(s), K, bias=dev(c["bias"]),
+                          out_dtype=torch.float32)
+    assert w4.last_linear_kernel() == expect
+    yr, bound = O.linear(c["x"], codes, O.expand_channel_scales(s, K), K, c["bias"])
+    ok, worst = O.check_linear(y.cpu().numpy().astype(np.float64), yr, bound)
+    assert ok, worst
+    yb = w4.linear_channel(bf16_dev(c["x_bits"]), dev(codes), dev(s), K, bias=dev(c["bias"]))
+    ok, worst = O.check_linear(yb.float().cpu().numpy().astype(np.float64), yr, bound)
+    assert ok, worst
+
+
+def test_linear_channel_one_hot_closed_form(w4):
+    """x = e_k picks column k: y = q[:, k] * s + b, computed exactly by the decode kernel
+    (one nonzero product per row, one scale multiply, one bias add, all in fp32)."""
+    N, K = 300, 4096
+    c = workloads.linear_case(4242, 1, N, K)
+    q, s = O.quantize_rtn_channel(c["W"])
+    codes = O.pack_nibbles(q)
+    for k in (0, 1, 4095, 1234):
+        xb = np.zeros((1, K), np.uint16)
+        xb[0, k] = 0x3F80  # 1.0
+        y = w4.linear_channel(bf16_dev(xb), dev(codes), dev(s), K, bias=dev(c["bias"]), out_dtype=torch.float32)
+        assert w4.last_linear_kernel() == "gemv_tma_channel"
+        want = (q[:, k].astype(np.float32) * s).astype(np.float32) + c["bias"]
+        assert np.array_equal(y.cpu().numpy()[0], want.astype(np.float32))
+
+
+def test_linear_channel_requires_workspace_off_the_decode_path(w4):
+    import ctypes
+    M, N, K = 20, 64, 1024
+    c = workloads.linear_case(7, M, N, K)
+    q, s = O.quantize_rtn_channel(c["W"])
+    x, cd, sd = bf16_dev(c["x_bits"]), dev(O.pack_nibbles(q)), dev(s)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    need = int(w4.lib.w4_linear_channel_workspace_bytes(M, N, K))
+    assert need >= N * (K // 32) * 4
+    st = w4.lib.w4_linear_channel(w4._ptr(x), M, w4._ptr(cd), w4._ptr(sd), N, K, None, w4._ptr(y), 0, None, 0,
+                                  w4._stream())
+    assert w4.STATUS[st] == "WORKSPACE"
+    assert int(w4.lib.w4_linear_channel_workspace_bytes(1, N, K)) == 0

@@ -34,7 +34,7 @@ EXPORTS = (
     "w4_set_weight_prefetch", "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
     "w4_dequantize_q4_0", "w4_linear_q4_0", "w4_linear_backward_x_workspace_bytes", "w4_linear_backward_x",
     "w4_quantize_rtn_channel", "w4_expand_channel_scales", "w4_lora_merge", "w4_selftest_wait_timeout",
-    "w4_last_linear_kernel",
+    "w4_last_linear_kernel", "w4_linear_channel_workspace_bytes", "w4_linear_channel",
 )
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -64,6 +64,8 @@ _SIGS = {
     "w4_lora_merge": [_vp, _vp, _i64, _i64, _vp, _vp, _i64, ctypes.c_float, _vp, _vp, _vp, _vp],
     "w4_selftest_wait_timeout": [ctypes.c_uint64, _vp],
     "w4_last_linear_kernel": [],
+    "w4_linear_channel_workspace_bytes": [_i64, _i64, _i64],
+    "w4_linear_channel": [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _vp, _i32, _vp, _sz, _vp],
 }
 _lib = None
 
@@ -84,6 +86,7 @@ def _load():
         handle.w4_linear_workspace_bytes.restype = ctypes.c_size_t
         handle.w4_linear_asym_workspace_bytes.restype = ctypes.c_size_t
         handle.w4_linear_backward_x_workspace_bytes.restype = ctypes.c_size_t
+        handle.w4_linear_channel_workspace_bytes.restype = ctypes.c_size_t
         handle.w4_status_string.restype = ctypes.c_char_p
         handle.w4_last_linear_kernel.restype = ctypes.c_char_p
         _lib = handle
@@ -194,6 +197,29 @@ def lora_merge(codes: torch.Tensor, scales: torch.Tensor, K: int, lora_b_t: torc
                                  float(alpha_over_rank), _ptr(co), _ptr(so), _ptr(status), _stream()),
            "w4_lora_merge")
     return co, so
+
+
+def linear_channel(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, K: int | None = None,
+                   bias: torch.Tensor | None = None, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """``y = x . dequant(W)^T + bias`` for a per-channel weight (``scales`` float32 ``[N]``)."""
+    _need_cuda(x, codes, scales, bias, out, workspace)
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    if scales.dtype != torch.float32 or scales.dim() != 1:
+        raise ValueError("scales must be a 1-D float32 tensor (one per row)")
+    M, Kx = x.shape
+    K = Kx if K is None else K
+    if K != Kx:
+        raise ValueError("x width does not match K")
+    N = codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    need = int(_load().w4_linear_channel_workspace_bytes(M, N, K))
+    ws, wsb = _workspace(M, N, K, x.device, workspace, need)
+    _check(_load().w4_linear_channel(_ptr(x), M, _ptr(codes), _ptr(scales), N, K, _ptr(bias), _ptr(out),
+                                     DTYPES[out.dtype], _ptr(ws), wsb, _stream()), "w4_linear_channel")
+    return out
 
 
 def expand_channel_scales(scales: torch.Tensor, K: int) -> torch.Tensor:

@@ -53,7 +53,7 @@ constexpr int kScaleBox = kRowsPerBlock * 32 * 4;          // 2 KB: 32 scales = 
 // shared memory a second CTA would need, so the warps come from one CTA), else 8. A stage
 // holds one k-tile per consumer warp.
 constexpr int warps_for(int nt) { return nt == 1 ? 16 : kWarps; }
-constexpr int stage_bytes(int w) { return w * kCodeBox + (w / 4) * kScaleBox; }
+constexpr int stage_bytes(int w, bool ch = false) { return w * kCodeBox + (ch ? 0 : (w / 4) * kScaleBox); }
 // Several activation rows: a reducer warp adds the consumer warps' row-block sums, so the
 // consumers never wait on each other (a row block is one or two stages there). One row: the
 // consumers meet at a named barrier per row block and one of them adds (measured 1-3% faster
@@ -97,9 +97,11 @@ struct TmaGemvParams {
   int y_dtype;
   int prefetch;    // stream codes and scales before the grid dependency resolves
   int boxes3d;     // 1: one 3-D box per stage for the codes and one for the scales
+  int channel;     // 1: one scale per row (scales [N]); applied once to the row's sum
 };
 
 __device__ __forceinline__ void store_y(const TmaGemvParams &p, int64_t m, int64_t n, float v) {
+  if (p.channel) v *= __ldg(p.scales + n);  // per-channel: the row's sum of code * x, scaled once
   if (p.bias) v += __ldcg(p.bias + n);
   if (p.y_dtype == W4_F32)
     static_cast<float *>(p.y)[m * p.N + n] = v;
@@ -188,13 +190,15 @@ __device__ __forceinline__ void unpack_asym(uint32_t w, uint32_t nzz, uint32_t (
 
 // NT = 0: M = 1, x broadcast to every MMA column. NT = 1, 2: up to 8 NT activation rows,
 // one per MMA column of each n-tile. ASYM: unsigned codes sorted by group (act-order),
-// per-(row, group) scale and zero point read through a per-CTA group table.
-template <int NT, bool ASYM>
+// per-(row, group) scale and zero point read through a per-CTA group table. CH: symmetric
+// codes with one scale per row (per-channel): the stages carry codes only, the group sums
+// are added unscaled and the row's scale multiplies its final sum.
+template <int NT, bool ASYM, bool CH>
 __global__ void __launch_bounds__(block_threads(NT), NT == 0 ? 2 : 1)
     gemv_tma_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
                     const __grid_constant__ CUtensorMap tm_zeros, const TmaGemvParams p, int32_t *err) {
   constexpr int W = warps_for(NT);            // consumer warps = k-tiles per stage
-  constexpr int SB = stage_bytes(W);          // bytes per stage
+  constexpr int SB = stage_bytes(W, CH);      // bytes per stage
   constexpr int kTok = NT == 0 ? 1 : 8 * NT;  // token slots of the reduction buffer
   constexpr int kAcc = NT == 0 ? 1 : NT;
   extern __shared__ uint8_t smem_raw[];
@@ -281,14 +285,15 @@ __global__ void __launch_bounds__(block_threads(NT), NT == 0 ? 2 : 1)
           // whole-stage boxes; k-tiles past the row end read as zeros (and count as bytes)
           mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(SB));
           tma_load_3d_hint(st, &tm_codes, 0, row, kt0, &full[slot], pol);
-          tma_load_3d_hint(st + W * kCodeBox, &tm_scales, 0, row, kt0 / 4, &full[slot], pol);
+          if (!CH) tma_load_3d_hint(st + W * kCodeBox, &tm_scales, 0, row, kt0 / 4, &full[slot], pol);
         } else {
-          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox + nsb * kScaleBox));
+          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(nkt * kCodeBox + (CH ? 0 : nsb * kScaleBox)));
           for (int j = 0; j < nkt; ++j)
             tma_load_2d_hint(st + j * kCodeBox, &tm_codes, (kt0 + j) * kKtileCodeBytes, row, &full[slot], pol);
-          for (int b = 0; b < nsb; ++b)
-            tma_load_2d_hint(st + W * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
-                        &full[slot], pol);
+          if (!CH)
+            for (int b = 0; b < nsb; ++b)
+              tma_load_2d_hint(st + W * kCodeBox + b * kScaleBox, &tm_scales, (kt0 + 4 * b) * 8, row,
+                               &full[slot], pol);
         }
         issued = i + 1;
         if (++kc == p.SPR) {
@@ -506,7 +511,28 @@ __global__ void __launch_bounds__(block_threads(NT), NT == 0 ? 2 : 1)
       uint32_t w[4][4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) ldsm_x4(cb + ld_off[q], w[q]);
-      if (!ASYM) {
+      if (!ASYM && CH) {
+        // per-channel: the k-tile's group sums added unscaled (the row's scale comes last)
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          uint32_t a[4], b[4];
+          unpack_signed(w[jj >> 1][(jj & 1) * 2], a);      // row g
+          unpack_signed(w[jj >> 1][(jj & 1) * 2 + 1], b);  // row g + 8
+#pragma unroll
+          for (int j = 0; j < kAcc; ++j) {
+            const uint4 xf = (NT == 0 || xok[j]) ? xrow[j][kt * 32 + 4 * jj] : make_uint4(0u, 0u, 0u, 0u);
+            float d[4];
+            mma_first(d, a[0], b[0], a[1], b[1], xf.x, xf.y);
+            mma_next(d, a[2], b[2], a[3], b[3], xf.z, xf.w);
+            acc[j][0] += d[0];
+            acc[j][2] += d[2];
+            if (NT != 0) {
+              acc[j][1] += d[1];
+              acc[j][3] += d[3];
+            }
+          }
+        }
+      } else if (!ASYM) {
         const uint8_t *sp = smem + slot * SB + sbox;
         const uint4 sg0 = *reinterpret_cast<const uint4 *>(sp + s_lo);
         const uint4 sg1 = *reinterpret_cast<const uint4 *>(sp + s_hi);
@@ -738,14 +764,15 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
     return false;  // act-order codes must be sorted by group (w4_asym_prepare)
   if (lp.K % 128 != 0 || lp.N > 0x7fffffffLL) return false;  // TMA: 16-byte row strides, int32 rows
   if (lp.y_dtype != W4_BF16 && lp.y_dtype != W4_F32) return false;
+  if (lp.channel && lp.asym) return false;
   const uintptr_t a = reinterpret_cast<uintptr_t>(lp.codes) | reinterpret_cast<uintptr_t>(lp.x) |
-                      (lp.asym ? 0 : reinterpret_cast<uintptr_t>(lp.scales));
+                      ((lp.asym || lp.channel) ? 0 : reinterpret_cast<uintptr_t>(lp.scales));
   if (a % 16 != 0) return false;
   const int64_t KT = (lp.K + 255) / 256;
   const int64_t x_stride = KT * 512 + 64;  // the 64 bytes keep two rows of a lane quad on distinct banks
   const int64_t tok = lp.M == 1 ? 1 : (lp.M <= 8 ? 8 : 16);
   const int W = warps_for(lp.M == 1 ? 0 : (lp.M <= 8 ? 1 : 2));
-  const int64_t SB = stage_bytes(W);
+  const int64_t SB = stage_bytes(W, lp.channel != 0);
   const int64_t red_floats = W * tok * kRowsPerBlock;
   const int64_t gtab_bytes = lp.asym ? KT * 10 * 4 : 0;
   const int64_t fixed = kAlignSlack + lp.M * x_stride + 2 * red_floats * 4 + gtab_bytes + kBarBytes;
@@ -760,7 +787,10 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   // ring a CTA of several row blocks requests most of its rows at once; every CTA's first
   // stage then lands late and compute overlaps the stream worse ((14336,4096): 8.6 us with
   // 3 stages, 9.7 us with 5; the other shapes unchanged).
-  if (lp.M == 1 && !lp.asym && S > 3) S = 3;
+  // Per-channel stages carry codes only (16 KB): five of them in flight measured best for
+  // the decode step (23.2 us with three or four, 21.8 with five, 22.0 with six).
+  const int64_t s_cap = lp.channel ? 5 : 3;
+  if (lp.M == 1 && !lp.asym && S > s_cap) S = s_cap;
   if (S < 2) return false;
   q->x = lp.x;
   q->bias = lp.bias;
@@ -783,6 +813,7 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   q->y_dtype = lp.y_dtype;
   q->prefetch = 0;
   q->boxes3d = 0;
+  q->channel = lp.channel;
   q->asym_staged = 0;
   q->x_sorted = 0;
   *smem = static_cast<int>(fixed + S * SB);
@@ -790,7 +821,7 @@ bool make_params(const LinearParams &lp, TmaGemvParams *q, int *smem, int *ctas_
   return true;
 }
 
-template <int NT, bool ASYM>
+template <int NT, bool ASYM, bool CH>
 cudaError_t ensure_smem_attr() {
   static std::mutex mu;
   static bool done[64] = {};
@@ -800,17 +831,17 @@ cudaError_t ensure_smem_attr() {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (!done[dev]) {
-    e = cudaFuncSetAttribute(gemv_tma_kernel<NT, ASYM>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    e = cudaFuncSetAttribute(gemv_tma_kernel<NT, ASYM, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
     if (e != cudaSuccess) return e;
     done[dev] = true;
   }
   return cudaSuccess;
 }
 
-template <int NT, bool ASYM>
+template <int NT, bool ASYM, bool CH = false>
 cudaError_t launch_typed(const CUtensorMap &mc, const CUtensorMap &ms, const CUtensorMap &mz, const TmaGemvParams &q,
                          int smem, int grid, int32_t *err, cudaStream_t stream) {
-  cudaError_t e = ensure_smem_attr<NT, ASYM>();
+  cudaError_t e = ensure_smem_attr<NT, ASYM, CH>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -822,7 +853,7 @@ cudaError_t launch_typed(const CUtensorMap &mc, const CUtensorMap &ms, const CUt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_tma_kernel<NT, ASYM>, mc, ms, mz, q, err);
+  return cudaLaunchKernelEx(&cfg, gemv_tma_kernel<NT, ASYM, CH>, mc, ms, mz, q, err);
 }
 
 }  // namespace
@@ -874,6 +905,15 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bf
                                    kRowsPerBlock, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     if (!q.asym_staged) ms = mz = mc;  // unused
+  } else if (lp.channel) {
+    // per-channel: codes only (one 3-D box per stage when the rows hold whole stages of k-tiles)
+    q.boxes3d = lp.K % 1024 == 0 &&
+                make_map_3d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, kKtileCodeBytes, lp.N, P / kKtileCodeBytes,
+                            P, kKtileCodeBytes, kKtileCodeBytes, kRowsPerBlock, W, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!q.boxes3d && !make_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, lp.codes, P, lp.N, P, kKtileCodeBytes,
+                                   kRowsPerBlock, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    ms = mz = mc;  // unused
   } else {
     // 3-D boxes need whole 256-column tiles of codes and whole 1024-column quads of scales in
     // every row (a box never reaches past a row's end into the next row)
@@ -900,6 +940,11 @@ cudaError_t launch_gemv_tma(const LinearParams &lp, bool prefetch, const __nv_bf
     if (lp.M == 1) return launch_typed<0, true>(mc, ms, mz, q, smem, gi, err, stream);
     if (lp.M <= 8) return launch_typed<1, true>(mc, ms, mz, q, smem, gi, err, stream);
     return launch_typed<2, true>(mc, ms, mz, q, smem, gi, err, stream);
+  }
+  if (lp.channel) {
+    if (lp.M == 1) return launch_typed<0, false, true>(mc, ms, mz, q, smem, gi, err, stream);
+    if (lp.M <= 8) return launch_typed<1, false, true>(mc, ms, mz, q, smem, gi, err, stream);
+    return launch_typed<2, false, true>(mc, ms, mz, q, smem, gi, err, stream);
   }
   if (lp.M == 1) return launch_typed<0, false>(mc, ms, mz, q, smem, gi, err, stream);
   if (lp.M <= 8) return launch_typed<1, false>(mc, ms, mz, q, smem, gi, err, stream);

@@ -397,6 +397,53 @@ w4_status w4_quantize_rtn_channel(const float *W, int64_t N, int64_t K, uint8_t 
   return W4_OK;
 }
 
+size_t w4_linear_channel_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  // none for the per-row-scale decode kernel (M <= 16, K a multiple of 128, aligned x and
+  // codes); otherwise the scales expanded to the group layout [N, ceil(K/32)] floats
+  if (M >= 1 && M <= 16 && K % 128 == 0) return 0;
+  if (N < 1 || K < 1) return 0;
+  return static_cast<size_t>(((N * ((K + 31) / 32) * 4 + 255) / 256) * 256);
+}
+
+w4_status w4_linear_channel(const void *x, int64_t M, const uint8_t *codes, const float *scales, int64_t N,
+                            int64_t K, const float *bias, void *y, w4_dtype y_dtype, void *workspace,
+                            size_t workspace_bytes, w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_linear_channel");
+  if (!x || !codes || !scales || !y) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || M < 1 || M > kMaxRows) return W4_ERR_SHAPE;
+  if (y_dtype != W4_BF16 && y_dtype != W4_F32) return W4_ERR_DTYPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  w4i::LinearParams p{};
+  p.x = static_cast<const __nv_bfloat16 *>(x);
+  p.codes = codes;
+  p.scales = scales;
+  p.bias = bias;
+  p.y = y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.y_dtype = y_dtype;
+  p.channel = 1;
+  if (w4i::gemv_tma_supports(p)) {
+    int32_t *err = nullptr;
+    const w4_status st = symbol_ptr(&err, g_device_error);
+    if (st != W4_OK) return st;
+    const cudaError_t e =
+        w4i::launch_gemv_tma(p, g_weight_prefetch.load(std::memory_order_relaxed) != 0, nullptr, err, s);
+    t_last_kernel = "gemv_tma_channel";
+    return e == cudaSuccess ? W4_OK : cuda_fail(e);
+  }
+  // other shapes: the row scales expanded to the group layout in the workspace, then the
+  // group-32 linear
+  const size_t need = static_cast<size_t>(N * ((K + 31) / 32) * 4);
+  if (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256) return W4_ERR_WORKSPACE;
+  cudaError_t e = w4i::launch_expand_channel_scales(scales, N, K, static_cast<float *>(workspace), s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  p.channel = 0;
+  p.scales = static_cast<const float *>(workspace);
+  return run_linear(p, nullptr, 0, s);
+}
+
 w4_status w4_expand_channel_scales(const float *scales, int64_t N, int64_t K, float *scales_out,
                                    w4_stream_t stream) {
   const NvtxRange nvtx_range("w4_expand_channel_scales");

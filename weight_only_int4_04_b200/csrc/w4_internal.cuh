@@ -28,6 +28,7 @@ struct LinearParams {
   int n_groups;            // asym only
   int y_dtype;             // W4_BF16 or W4_F32
   int asym;                // 0 = symmetric signed codes, 1 = asymmetric unsigned codes
+  int channel;             // symmetric only: 1 = one scale per row, scales [N] (per-channel)
 };
 
 // Each launcher enqueues on `stream` and returns the launch error (cudaSuccess or not).
