@@ -97,3 +97,40 @@ def test_backward_x_is_adjoint_of_linear(w4):
     # sum over (m, n, k) of |x w dy|: each side is within 4e-3 of it
     scale = float(((np.abs(c["x"].astype(np.float64)) @ np.abs(w).T) * np.abs(dy)).sum())
     assert abs(lhs - rhs) <= 8e-3 * scale
+
+
+# the tensor-core kernel (2 <= M, K a multiple of 128, N a multiple of 8): ragged 32-row steps,
+# several 16-row token tiles, row splits, the full-size shape
+MMA_CASES = [(2, 64, 128), (5, 1000, 384), (16, 14336, 4096), (64, 2048, 1024), (17, 8, 256), (40, 3000, 640)]
+
+
+@pytest.mark.parametrize("MNK", MMA_CASES, ids=[f"M{m}_N{n}_K{k}" for m, n, k in MMA_CASES])
+def test_backward_x_tensor_core(w4, MNK):
+    M, N, K = MNK
+    codes, s, dy_bits, dy = case(M, N, K, M * 17 + N + K)
+    dxr, bound = O.linear_backward_x(dy, codes, s, K)
+    ddy, dc, ds = bf16_dev(dy_bits), dev(codes), dev(s)
+    for dt in (torch.float32, torch.bfloat16):
+        dx = w4.linear_backward_x(ddy, dc, ds, K, out_dtype=dt)
+        check(dx.float().cpu().numpy().astype(np.float64), dxr, bound, (M, N, K, str(dt)))
+    a = w4.linear_backward_x(ddy, dc, ds, K, out_dtype=torch.float32)
+    b = w4.linear_backward_x(ddy, dc, ds, K, out_dtype=torch.float32)
+    assert torch.equal(a, b)  # fixed-order split sums: bitwise repeatable
+
+
+def test_backward_x_tensor_core_one_hot(w4):
+    """One-hot upstream rows pick one weight row. The tensor-core kernel carries each weight
+    as a pair of bf16 values whose sum is within 2^-16 of the fp32 dequantized weight, so dx
+    must match that row to 2^-15 relative -- far inside the linear tolerance, and far from
+    what a single bf16 weight (2^-8) would give."""
+    M, N, K = 4, 96, 512
+    codes, s, _, _ = case(M, N, K, 12)
+    w = O.dequantize(codes, s, K, "f32").astype(np.float64)
+    rows = [0, 31, 32, 95]
+    dy = np.zeros((M, N), np.float32)
+    for m, n in enumerate(rows):
+        dy[m, n] = 1.0
+    dx = w4.linear_backward_x(bf16_dev(O.f32_to_bf16_bits(dy)), dev(codes), dev(s), K, out_dtype=torch.float32)
+    got = dx.cpu().numpy().astype(np.float64)
+    for m, n in enumerate(rows):
+        assert np.all(np.abs(got[m] - w[n]) <= 2.0**-15 * np.abs(w[n])), (m, n)

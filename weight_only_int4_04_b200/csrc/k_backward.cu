@@ -16,8 +16,24 @@
 //     token. The warps' sums meet in shared memory in a fixed order; when the rows are split
 //     over several CTAs each writes its partial sums to the workspace and
 //     bwd_x_reduce_kernel adds the splits in a fixed order (deterministic results).
+//   * bwd_x_mma_kernel (2 <= M, K a multiple of 128, N a multiple of 8, 4-byte aligned codes
+//     and scales, 16-byte aligned dy): tensor cores. A CTA owns 128 columns, a slice of rows
+//     and 16 upstream rows. Per step of 32 weight rows its threads dequantize one code word
+//     each: the fp32 weight w = fl32(q * s) is written as two bf16 tiles, hi = bf16(w) and
+//     lo = bf16(w - hi) (w - hi is exact in fp32; hi + lo is within 2^-16 |w| of w, so the
+//     contraction carries fp32-like weights and the output rounding keeps the tolerance; one
+//     bf16 weight alone could cost 2^-8 per term), with 16-byte chunks XOR-swizzled by the
+//     row so that both the stores and the transposing loads are conflict-free; the upstream
+//     rows go to a padded tile. ldmatrix gives the A fragments (upstream rows x weight
+//     rows), ldmatrix.trans the B fragments (weight rows x columns: the contraction axis is the
+//     weight's row axis, which the packed codes do not pair), and mma.sync m16n8k16 (bf16 in,
+//     fp32 accumulate) does the contraction, two MMAs (hi, lo) per fragment into one
+//     accumulator; warp w owns columns 32w .. 32w+31. Two buffers,
+//     one barrier per step; the next step's codes, scales and upstream values are in flight
+//     while the current step multiplies. Row splits meet in bwd_x_reduce_kernel as above.
 //   * bwd_x_plain_kernel: any K, one thread per (token, column), rows in order.
-#include "w4_internal.cuh"
+#include "w4_mma.cuh"
+#include "w4_tc.cuh"
 
 namespace w4i {
 
@@ -28,6 +44,7 @@ constexpr int kBwdWarps = 8;
 constexpr int kBwdTargetCtas = 592;  // four per SM on a 148-SM part; sets the row split
 constexpr int kBwdStageRows = 1024;  // rows whose upstream gradient is staged in shared memory at once
 constexpr int64_t kBwdMinRows = 64;  // rows per split at least
+constexpr int64_t kBwdMmaMinM = 2;   // upstream rows from which the tensor-core kernel serves
 
 __device__ __forceinline__ uint32_t ld_stream_u32(const uint32_t *p) {
   uint32_t v;
@@ -219,6 +236,164 @@ __global__ void __launch_bounds__(32 * kBwdWarps) bwd_x_wide_kernel(const __nv_b
   }
 }
 
+constexpr int kMmaCols = 128;   // columns per CTA (four warps x 32)
+constexpr int kMmaRows = 32;    // weight rows per step
+constexpr int kMmaTok = 16;     // upstream rows per CTA (the MMA's M)
+constexpr int kMmaThreads = 128;
+constexpr int kWtPitch = kMmaCols * 2;  // bytes per row of the bf16 weight tile
+constexpr int kDyPitch = 80;            // 32 bf16 + 16 bytes: conflict-free ldmatrix rows
+
+// Eight nibbles of one code word -> the fp32 weights fl32(q * s) of columns 8t .. 8t+7 as two
+// bf16 words per pair: hi = bf16(w), lo = bf16(w - hi), both packed in column order.
+__device__ __forceinline__ void dequant_word_split(uint32_t w, float s, uint4 &hi, uint4 &lo) {
+  const uint32_t el = lop3_and_xor(w, 0x0F0F0F0Fu, 0x08080808u);       // even columns, nibble ^ 8
+  const uint32_t od = lop3_and_xor(w >> 4, 0x0F0F0F0Fu, 0x08080808u);  // odd columns
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    // 2^23 + (q + 8) in both halves of an fp32 pair, minus 2^23 + 8: exactly q
+    const float qe = __uint_as_float(prmt(el, 0x00004B00u, 0x5440u | i)) - 8388616.0f;
+    const float qo = __uint_as_float(prmt(od, 0x00004B00u, 0x5440u | i)) - 8388616.0f;
+    const float we = __fmul_rn(qe, s), wo = __fmul_rn(qo, s);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(h[i]) : "f"(wo), "f"(we));
+    const float re = we - __uint_as_float(h[i] << 16), ro = wo - __uint_as_float(h[i] & 0xFFFF0000u);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(l[i]) : "f"(ro), "f"(re));
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&d)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_acc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloat16 *__restrict__ dy,
+                                                                const uint8_t *__restrict__ codes,
+                                                                const float *__restrict__ scales, float *part,
+                                                                void *dx, int dx_dtype, int64_t M, int64_t N,
+                                                                int64_t K, int64_t rows_per_split, int splits) {
+  __shared__ __align__(128) uint8_t wt[2][2][kMmaRows * kWtPitch];  // [buffer][hi, lo]
+  __shared__ __align__(128) uint8_t dys[2][kMmaTok * kDyPitch];
+  const int tid = static_cast<int>(threadIdx.x), warp = tid >> 5, lane = tid & 31;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kMmaCols;
+  const int split = static_cast<int>(blockIdx.y);
+  const int64_t m0 = static_cast<int64_t>(blockIdx.z) * kMmaTok;
+  const int64_t n_begin = static_cast<int64_t>(split) * rows_per_split;
+  const int64_t n_end = (n_begin + rows_per_split < N) ? n_begin + rows_per_split : N;
+  const int64_t P = K / 2, G = K / 32;
+  // dequant role: code word c (columns 8c .. 8c+7 of the tile) of rows rb, rb + 8, rb + 16, rb + 24
+  const int c = tid & 15, rb = tid >> 4;
+  const uint32_t *cw_base = reinterpret_cast<const uint32_t *>(codes + k0 / 2) + c;
+  const float *sc_base = scales + k0 / 32 + (c >> 2);
+  // upstream role (threads 0..63): row tok of the 16, eight weight rows q8 .. q8+7 of the step
+  const int tok = tid >> 2, q8 = (tid & 3) * 8;
+  const bool dy_row = tid < 64 && m0 + tok < M;
+  const __nv_bfloat16 *dy_base = dy + (m0 + tok) * N + q8;
+
+  uint32_t cw[4];
+  float sc[4];
+  uint4 dv = make_uint4(0u, 0u, 0u, 0u);
+  auto fetch = [&](int64_t n0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t n = n0 + rb + 8 * j;
+      const bool ok = n < n_end;
+      cw[j] = ok ? __ldg(cw_base + n * (P / 4)) : 0u;  // rows past the slice: code 0, scale 0
+      sc[j] = ok ? __ldg(sc_base + n * G) : 0.0f;
+    }
+    if (dy_row && n0 + q8 < n_end) dv = __ldg(reinterpret_cast<const uint4 *>(dy_base + n0));
+    else dv = make_uint4(0u, 0u, 0u, 0u);
+  };
+  auto put = [&](int buf) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int r = rb + 8 * j;
+      uint4 vh, vl;
+      dequant_word_split(cw[j], sc[j], vh, vl);
+      const int off = r * kWtPitch + ((c ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4 *>(&wt[buf][0][off]) = vh;
+      *reinterpret_cast<uint4 *>(&wt[buf][1][off]) = vl;
+    }
+    if (tid < 64) *reinterpret_cast<uint4 *>(&dys[buf][tok * kDyPitch + (tid & 3) * 16]) = dv;
+  };
+
+  // per-lane ldmatrix addresses (offsets inside a buffer)
+  // A (upstream rows x weight rows, row-major): matrix i = lane >> 3: rows (l & 7) + 8 (i & 1),
+  // columns 8 (i >> 1) .. of the 16-row half h
+  const int li = lane >> 3, lr = lane & 7;
+  const uint32_t a_off = static_cast<uint32_t>((lr + 8 * (li & 1)) * kDyPitch + 16 * (li >> 1));
+  // B (weight rows x columns, transposed on load): matrix i: rows (l & 7) + 8 (i & 1) of the
+  // half, 16-byte chunk 4 warp + pair + (i >> 1)
+  const int b_row = lr + 8 * (li & 1);
+
+  float acc[4][4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+
+  const int steps = n_end > n_begin ? static_cast<int>((n_end - n_begin + kMmaRows - 1) / kMmaRows) : 0;
+  if (steps > 0) {
+    fetch(n_begin);
+    put(0);
+  }
+  for (int it = 0; it < steps; ++it) {
+    const int buf = it & 1;
+    if (it + 1 < steps) fetch(n_begin + static_cast<int64_t>(it + 1) * kMmaRows);
+    __syncthreads();  // this buffer's tiles are written; the other one's readers are done
+    const uint32_t wbase = smem_u32(&wt[buf][0][0]);
+    constexpr uint32_t kLoTile = kMmaRows * kWtPitch;  // lo tile follows the hi tile
+    const uint32_t dbase = smem_u32(&dys[buf][0]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t a[4];
+      ldsm_x4(dbase + a_off + 32u * h, a);
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const int row = 16 * h + b_row;
+        const int chunk = 4 * warp + 2 * pr + (li >> 1);
+        const uint32_t boff = wbase + static_cast<uint32_t>(row * kWtPitch + ((chunk ^ (row & 7)) << 4));
+        uint32_t b[4], bl[4];
+        ldsm_x4_trans(boff, b);
+        ldsm_x4_trans(boff + kLoTile, bl);
+        mma_acc(acc[2 * pr], a, b[0], b[1]);
+        mma_acc(acc[2 * pr + 1], a, b[2], b[3]);
+        mma_acc(acc[2 * pr], a, bl[0], bl[1]);
+        mma_acc(acc[2 * pr + 1], a, bl[2], bl[3]);
+      }
+    }
+    if (it + 1 < steps) put(buf ^ 1);
+  }
+
+  // acc[j]: upstream rows g, g + 8 x columns 32 warp + 8 j + 2 t (+1)
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t kk = k0 + 32 * warp + 8 * j + 2 * t;
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int64_t m = m0 + g + 8 * hf;
+      if (m >= M) continue;
+      const float v0 = acc[j][2 * hf], v1 = acc[j][2 * hf + 1];
+      if (splits == 1) {
+        store_out(dx, dx_dtype, m * K + kk, v0);
+        store_out(dx, dx_dtype, m * K + kk + 1, v1);
+      } else {
+        float *dst = part + (static_cast<int64_t>(split) * M + m) * K + kk;
+        dst[0] = v0;
+        dst[1] = v1;
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) bwd_x_reduce_kernel(const float *__restrict__ part, void *dx, int dx_dtype,
                                                            int64_t MK, int splits) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -267,6 +442,26 @@ int64_t bwd_splits(int64_t M, int64_t N, int64_t K) {
   return s;
 }
 
+// Row splits of the tensor-core kernel: about four CTAs per SM, whole 32-row steps.
+bool bwd_mma_shape(int64_t M, int64_t N, int64_t K) {
+  return M >= kBwdMmaMinM && K % kMmaCols == 0 && N % 8 == 0 && (M + kMmaTok - 1) / kMmaTok <= 65535;
+}
+
+int64_t bwd_mma_rows(int64_t M, int64_t N, int64_t K) {
+  const int64_t ctas = (K / kMmaCols) * ((M + kMmaTok - 1) / kMmaTok);
+  int64_t splits = (kBwdTargetCtas + ctas - 1) / ctas;
+  const int64_t max_splits = (N + kMmaRows - 1) / kMmaRows;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  const int64_t rows = (N + splits - 1) / splits;
+  return (rows + kMmaRows - 1) / kMmaRows * kMmaRows;
+}
+
+int64_t bwd_mma_splits(int64_t M, int64_t N, int64_t K) {
+  const int64_t rows = bwd_mma_rows(M, N, K);
+  return (N + rows - 1) / rows;
+}
+
 template <int TM>
 cudaError_t launch_tm(const __nv_bfloat16 *dy, const uint8_t *codes, const float *scales, float *part, void *dx,
                       int dx_dtype, int64_t M, int64_t N, int64_t K, int64_t splits, cudaStream_t stream) {
@@ -289,13 +484,32 @@ cudaError_t launch_tm(const __nv_bfloat16 *dy, const uint8_t *codes, const float
 
 size_t linear_backward_x_workspace(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < 1 || K % 8 != 0) return 0;
+  // the larger of the two kernels' needs: which one serves can depend on pointer alignment
   const int64_t s = bwd_splits(M, N, K);
-  return s > 1 ? static_cast<size_t>(s) * static_cast<size_t>(M) * static_cast<size_t>(K) * sizeof(float) : 0;
+  const int64_t s2 = bwd_mma_shape(M, N, K) ? bwd_mma_splits(M, N, K) : 1;
+  const int64_t sm = s > s2 ? s : s2;
+  return sm > 1 ? static_cast<size_t>(sm) * static_cast<size_t>(M) * static_cast<size_t>(K) * sizeof(float) : 0;
 }
 
 cudaError_t launch_linear_backward_x(const __nv_bfloat16 *dy, int64_t M, const uint8_t *codes, const float *scales,
                                      int64_t N, int64_t K, void *dx, int dx_dtype, void *workspace,
                                      size_t workspace_bytes, cudaStream_t stream) {
+  if (bwd_mma_shape(M, N, K) && bwd_fast(codes, scales, K) && reinterpret_cast<uintptr_t>(dy) % 16 == 0) {
+    const int64_t rows = bwd_mma_rows(M, N, K), splits = (N + rows - 1) / rows;
+    const size_t need_mma = splits > 1 ? static_cast<size_t>(splits * M * K) * sizeof(float) : 0;
+    if (need_mma == 0 || (workspace != nullptr && workspace_bytes >= need_mma)) {
+      const dim3 grid(static_cast<unsigned>(K / kMmaCols), static_cast<unsigned>(splits),
+                      static_cast<unsigned>((M + kMmaTok - 1) / kMmaTok));
+      bwd_x_mma_kernel<<<grid, kMmaThreads, 0, stream>>>(dy, codes, scales, static_cast<float *>(workspace), dx,
+                                                         dx_dtype, M, N, K, rows, static_cast<int>(splits));
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess || splits == 1) return e;
+      const int64_t MK = M * K;
+      bwd_x_reduce_kernel<<<static_cast<unsigned>((MK + 255) / 256), 256, 0, stream>>>(
+          static_cast<float *>(workspace), dx, dx_dtype, MK, static_cast<int>(splits));
+      return cudaGetLastError();
+    }
+  }
   const size_t need = linear_backward_x_workspace(M, N, K);
   const bool chunks_fit = (M + bwd_tm(M) - 1) / bwd_tm(M) <= 65535;  // grid z of the streaming kernel
   if (bwd_fast(codes, scales, K) && chunks_fit && (need == 0 || (workspace != nullptr && workspace_bytes >= need))) {
