@@ -18,8 +18,9 @@
 //     bwd_x_reduce_kernel adds the splits in a fixed order (deterministic results).
 //   * bwd_x_mma_kernel (2 <= M, K a multiple of 128, N a multiple of 8, 4-byte aligned codes
 //     and scales, 16-byte aligned dy): tensor cores. A CTA owns 128 columns, a slice of rows
-//     and 16 upstream rows. Per step of 32 weight rows its threads dequantize one code word
-//     each: the fp32 weight w = fl32(q * s) is written as two bf16 tiles, hi = bf16(w) and
+//     and 16 upstream rows. Per step of 32 weight rows each thread dequantizes one 32-column
+//     group of one row (one 16-byte code load, one scale): the fp32 weight w = fl32(q * s) is
+//     written as two bf16 tiles, hi = bf16(w) and
 //     lo = bf16(w - hi) (w - hi is exact in fp32; hi + lo is within 2^-16 |w| of w, so the
 //     contraction carries fp32-like weights and the output rounding keeps the tolerance; one
 //     bf16 weight alone could cost 2^-8 per term), with 16-byte chunks XOR-swizzled by the
@@ -29,8 +30,8 @@
 //     weight's row axis, which the packed codes do not pair), and mma.sync m16n8k16 (bf16 in,
 //     fp32 accumulate) does the contraction, two MMAs (hi, lo) per fragment into one
 //     accumulator; warp w owns columns 32w .. 32w+31. Two buffers,
-//     one barrier per step; the next step's codes, scales and upstream values are in flight
-//     while the current step multiplies. Row splits meet in bwd_x_reduce_kernel as above.
+//     one barrier per step; the codes, scales and upstream values of the next two steps are in
+//     flight while the current step multiplies. Row splits meet in bwd_x_reduce_kernel as above.
 //   * bwd_x_plain_kernel: any K, one thread per (token, column), rows in order.
 #include "w4_mma.cuh"
 #include "w4_tc.cuh"
@@ -45,6 +46,7 @@ constexpr int kBwdTargetCtas = 592;  // four per SM on a 148-SM part; sets the r
 constexpr int kBwdStageRows = 1024;  // rows whose upstream gradient is staged in shared memory at once
 constexpr int64_t kBwdMinRows = 64;  // rows per split at least
 constexpr int64_t kBwdMmaMinM = 2;   // upstream rows from which the tensor-core kernel serves
+constexpr int64_t kBwdMmaTargetCtas = 888;  // six 128-thread CTAs per SM of a 148-SM part
 
 __device__ __forceinline__ uint32_t ld_stream_u32(const uint32_t *p) {
   uint32_t v;
@@ -244,20 +246,30 @@ constexpr int kWtPitch = kMmaCols * 2;  // bytes per row of the bf16 weight tile
 constexpr int kDyPitch = 80;            // 32 bf16 + 16 bytes: conflict-free ldmatrix rows
 
 // Eight nibbles of one code word -> the fp32 weights fl32(q * s) of columns 8t .. 8t+7 as two
-// bf16 words per pair: hi = bf16(w), lo = bf16(w - hi), both packed in column order.
-__device__ __forceinline__ void dequant_word_split(uint32_t w, float s, uint4 &hi, uint4 &lo) {
+// bf16 words per pair: hi = bf16(w), lo = bf16(w - hi), both packed in column order. Per column
+// pair: the nibble (xor 8) in the low byte of the fp32 2^23 (PRMT), one exact fp32x2 subtract of
+// 2^23 + 8 leaves q, one fp32x2 multiply by the scale rounds once; hi is widened back (PRMT /
+// LOP3) and the remainder w - hi (exact) is rounded to bf16.
+__device__ __forceinline__ void dequant_word_split(uint32_t w, uint64_t scale2, uint4 &hi, uint4 &lo) {
   const uint32_t el = lop3_and_xor(w, 0x0F0F0F0Fu, 0x08080808u);       // even columns, nibble ^ 8
   const uint32_t od = lop3_and_xor(w >> 4, 0x0F0F0F0Fu, 0x08080808u);  // odd columns
+  const uint64_t nb2 = neg_bias_pair(8u);
   uint32_t h[4], l[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    // 2^23 + (q + 8) in both halves of an fp32 pair, minus 2^23 + 8: exactly q
-    const float qe = __uint_as_float(prmt(el, 0x00004B00u, 0x5440u | i)) - 8388616.0f;
-    const float qo = __uint_as_float(prmt(od, 0x00004B00u, 0x5440u | i)) - 8388616.0f;
-    const float we = __fmul_rn(qe, s), wo = __fmul_rn(qo, s);
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(h[i]) : "f"(wo), "f"(we));
-    const float re = we - __uint_as_float(h[i] << 16), ro = wo - __uint_as_float(h[i] & 0xFFFF0000u);
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(l[i]) : "f"(ro), "f"(re));
+    const uint32_t fe = prmt(el, 0x00004B00u, 0x5440u | i);
+    const uint32_t fo = prmt(od, 0x00004B00u, 0x5440u | i);
+    uint64_t v = (static_cast<uint64_t>(fo) << 32) | fe;
+    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(nb2));
+    asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(scale2));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+        : "=r"(h[i])
+        : "f"(__uint_as_float(static_cast<uint32_t>(v >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(v))));
+    const uint64_t hw = (static_cast<uint64_t>(h[i] & 0xFFFF0000u) << 32) | prmt(h[i], 0u, 0x1044u);
+    asm("sub.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(hw));
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+        : "=r"(l[i])
+        : "f"(__uint_as_float(static_cast<uint32_t>(v >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(v))));
   }
   hi = make_uint4(h[0], h[1], h[2], h[3]);
   lo = make_uint4(l[0], l[1], l[2], l[3]);
@@ -290,40 +302,44 @@ __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloa
   const int64_t n_begin = static_cast<int64_t>(split) * rows_per_split;
   const int64_t n_end = (n_begin + rows_per_split < N) ? n_begin + rows_per_split : N;
   const int64_t P = K / 2, G = K / 32;
-  // dequant role: code word c (columns 8c .. 8c+7 of the tile) of rows rb, rb + 8, rb + 16, rb + 24
-  const int c = tid & 15, rb = tid >> 4;
-  const uint32_t *cw_base = reinterpret_cast<const uint32_t *>(codes + k0 / 2) + c;
-  const float *sc_base = scales + k0 / 32 + (c >> 2);
+  // dequant role: row r of the step, the 32 columns of group q of the tile (four code words,
+  // one 16-byte load, one scale)
+  const int r = tid >> 2, q = tid & 3;
+  const uint4 *cw_base = reinterpret_cast<const uint4 *>(codes + k0 / 2) + q;
+  const float *sc_base = scales + k0 / 32 + q;
   // upstream role (threads 0..63): row tok of the 16, eight weight rows q8 .. q8+7 of the step
   const int tok = tid >> 2, q8 = (tid & 3) * 8;
   const bool dy_row = tid < 64 && m0 + tok < M;
   const __nv_bfloat16 *dy_base = dy + (m0 + tok) * N + q8;
 
-  uint32_t cw[4];
-  float sc[4];
-  uint4 dv = make_uint4(0u, 0u, 0u, 0u);
-  auto fetch = [&](int64_t n0) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t n = n0 + rb + 8 * j;
-      const bool ok = n < n_end;
-      cw[j] = ok ? __ldg(cw_base + n * (P / 4)) : 0u;  // rows past the slice: code 0, scale 0
-      sc[j] = ok ? __ldg(sc_base + n * G) : 0.0f;
-    }
-    if (dy_row && n0 + q8 < n_end) dv = __ldg(reinterpret_cast<const uint4 *>(dy_base + n0));
-    else dv = make_uint4(0u, 0u, 0u, 0u);
+  struct Step {
+    uint4 cw;
+    float sc;
+    uint4 dv;
   };
-  auto put = [&](int buf) {
+  // rows past the slice: codes 0, scale 0, upstream 0
+  auto fetch = [&](Step &st, int64_t n0) {
+    const int64_t n = n0 + r;
+    const bool ok = n < n_end;
+    st.cw = ok ? __ldg(cw_base + n * (P / 16)) : make_uint4(0u, 0u, 0u, 0u);
+    st.sc = ok ? __ldg(sc_base + n * G) : 0.0f;
+    st.dv = (dy_row && n0 + q8 < n_end) ? __ldg(reinterpret_cast<const uint4 *>(dy_base + n0))
+                                        : make_uint4(0u, 0u, 0u, 0u);
+  };
+  auto put = [&](const Step &st, int buf) {
+    const uint64_t s2 = (static_cast<uint64_t>(__float_as_uint(st.sc)) << 32) | __float_as_uint(st.sc);
+    const uint32_t words[4] = {st.cw.x, st.cw.y, st.cw.z, st.cw.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int r = rb + 8 * j;
+      // the four lanes of a row start at different chunks: fewer bank conflicts on the stores
+      const int jj = (j + q) & 3;
       uint4 vh, vl;
-      dequant_word_split(cw[j], sc[j], vh, vl);
-      const int off = r * kWtPitch + ((c ^ (r & 7)) << 4);
+      dequant_word_split(words[jj], s2, vh, vl);
+      const int off = r * kWtPitch + (((4 * q + jj) ^ (r & 7)) << 4);
       *reinterpret_cast<uint4 *>(&wt[buf][0][off]) = vh;
       *reinterpret_cast<uint4 *>(&wt[buf][1][off]) = vl;
     }
-    if (tid < 64) *reinterpret_cast<uint4 *>(&dys[buf][tok * kDyPitch + (tid & 3) * 16]) = dv;
+    if (tid < 64) *reinterpret_cast<uint4 *>(&dys[buf][tok * kDyPitch + (tid & 3) * 16]) = st.dv;
   };
 
   // per-lane ldmatrix addresses (offsets inside a buffer)
@@ -340,17 +356,10 @@ __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloa
   for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
 
   const int steps = n_end > n_begin ? static_cast<int>((n_end - n_begin + kMmaRows - 1) / kMmaRows) : 0;
-  if (steps > 0) {
-    fetch(n_begin);
-    put(0);
-  }
-  for (int it = 0; it < steps; ++it) {
-    const int buf = it & 1;
-    if (it + 1 < steps) fetch(n_begin + static_cast<int64_t>(it + 1) * kMmaRows);
-    __syncthreads();  // this buffer's tiles are written; the other one's readers are done
+  auto multiply = [&](int buf) {
     const uint32_t wbase = smem_u32(&wt[buf][0][0]);
-    constexpr uint32_t kLoTile = kMmaRows * kWtPitch;  // lo tile follows the hi tile
     const uint32_t dbase = smem_u32(&dys[buf][0]);
+    constexpr uint32_t kLoTile = kMmaRows * kWtPitch;  // lo tile follows the hi tile
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t a[4];
@@ -369,7 +378,24 @@ __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloa
         mma_acc(acc[2 * pr + 1], a, bl[2], bl[3]);
       }
     }
-    if (it + 1 < steps) put(buf ^ 1);
+  };
+  // two steps in flight: step i's loads are issued two steps ahead of its multiply
+  Step sa, sb;
+  if (steps > 0) fetch(sa, n_begin);
+  if (steps > 1) fetch(sb, n_begin + kMmaRows);
+  if (steps > 0) put(sa, 0);
+  for (int it = 0; it < steps; it += 2) {
+    // even step: buffer 0 holds it; sb holds it + 1
+    if (it + 2 < steps) fetch(sa, n_begin + static_cast<int64_t>(it + 2) * kMmaRows);
+    __syncthreads();  // buffer 0 is written; buffer 1's readers (step it - 1) are done
+    multiply(0);
+    if (it + 1 >= steps) break;
+    put(sb, 1);
+    // odd step: buffer 1 holds it + 1; sa holds it + 2
+    if (it + 3 < steps) fetch(sb, n_begin + static_cast<int64_t>(it + 3) * kMmaRows);
+    __syncthreads();
+    multiply(1);
+    if (it + 2 < steps) put(sa, 0);
   }
 
   // acc[j]: upstream rows g, g + 8 x columns 32 warp + 8 j + 2 t (+1)
@@ -449,7 +475,7 @@ bool bwd_mma_shape(int64_t M, int64_t N, int64_t K) {
 
 int64_t bwd_mma_rows(int64_t M, int64_t N, int64_t K) {
   const int64_t ctas = (K / kMmaCols) * ((M + kMmaTok - 1) / kMmaTok);
-  int64_t splits = (kBwdTargetCtas + ctas - 1) / ctas;
+  int64_t splits = (kBwdMmaTargetCtas + ctas - 1) / ctas;
   const int64_t max_splits = (N + kMmaRows - 1) / kMmaRows;
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
@@ -494,7 +520,8 @@ size_t linear_backward_x_workspace(int64_t M, int64_t N, int64_t K) {
 cudaError_t launch_linear_backward_x(const __nv_bfloat16 *dy, int64_t M, const uint8_t *codes, const float *scales,
                                      int64_t N, int64_t K, void *dx, int dx_dtype, void *workspace,
                                      size_t workspace_bytes, cudaStream_t stream) {
-  if (bwd_mma_shape(M, N, K) && bwd_fast(codes, scales, K) && reinterpret_cast<uintptr_t>(dy) % 16 == 0) {
+  if (bwd_mma_shape(M, N, K) && bwd_fast(codes, scales, K) &&
+      (reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(codes)) % 16 == 0) {
     const int64_t rows = bwd_mma_rows(M, N, K), splits = (N + rows - 1) / rows;
     const size_t need_mma = splits > 1 ? static_cast<size_t>(splits * M * K) * sizeof(float) : 0;
     if (need_mma == 0 || (workspace != nullptr && workspace_bytes >= need_mma)) {
