@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(threads_for(BN), 1)
   uint64_t *acc_full = empty + STAGES;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *issued_sm = const_cast<int *>(abort_flag) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BM_W;
@@ -136,12 +137,11 @@ __global__ void __launch_bounds__(threads_for(BN), 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < KB; ++kb) {
+      int kb = 0;
+      for (; kb < KB; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = static_cast<uint32_t>(kb / STAGES) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, err)) break;
-        issued = kb + 1;
         mbar_arrive_expect_tx(&full_load[s], L::TX);
         tma_load_2d(smem + L::OFF_B + s * L::B_BYTES, &tmap_x, kb * BK, static_cast<int32_t>(m0), &full_load[s]);
         tma_load_2d(smem + L::OFF_C + s * C_BYTES, &tmap_codes, kb * (BK / 2), static_cast<int32_t>(n0),
@@ -155,9 +155,7 @@ __global__ void __launch_bounds__(threads_for(BN), 1)
           tma_load_2d(smem + L::OFF_Z + s * Z_BYTES, &tmap_zeros, gs & ~15, static_cast<int32_t>(n0), &full_load[s]);
         }
       }
-      // the copies issued land before the CTA may exit (see w4_sync.cuh, abort path)
-      for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
-        mbar_drain(&full_load[kb % STAGES], static_cast<uint32_t>(kb / STAGES) & 1u, err);
+      *issued_sm = kb;  // stages whose copies were issued (read on the abort path below)
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -178,9 +176,6 @@ __global__ void __launch_bounds__(threads_for(BN), 1)
         umma_commit(&empty[s]);
       }
       umma_commit(acc_full);
-      // every MMA issued has finished before the CTA frees its tensor memory (the epilogue
-      // stops waiting on an abort)
-      mbar_drain(acc_full, 0u, err);
     }
   } else {
     // ---- dequantize into the A stages ----
@@ -296,6 +291,15 @@ __global__ void __launch_bounds__(threads_for(BN), 1)
     }
   }
   tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // abort path (see w4_sync.cuh): the consumers stopped waiting, so the copies issued must
+    // land and every MMA must finish before the CTA frees its tensor memory and exits
+    const int issued = *issued_sm;
+    for (int kb = issued - STAGES < 0 ? 0 : issued - STAGES; kb < issued; ++kb)
+      mbar_drain(&full_load[kb % STAGES], static_cast<uint32_t>(kb / STAGES) & 1u, err);
+    mbar_drain(acc_full, 0u, err);
+  }
   __syncthreads();
   if (warp == 1) {
     __syncwarp();
