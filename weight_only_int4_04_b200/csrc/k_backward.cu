@@ -16,22 +16,22 @@
 //     token. The warps' sums meet in shared memory in a fixed order; when the rows are split
 //     over several CTAs each writes its partial sums to the workspace and
 //     bwd_x_reduce_kernel adds the splits in a fixed order (deterministic results).
-//   * bwd_x_mma_kernel (2 <= M, K a multiple of 128, N a multiple of 8, 4-byte aligned codes
-//     and scales, 16-byte aligned dy): tensor cores. A CTA owns 128 columns, a slice of rows
-//     and 16 upstream rows. Per step of 32 weight rows each thread dequantizes one 32-column
-//     group of one row (one 16-byte code load, one scale): the fp32 weight w = fl32(q * s) is
-//     written as two bf16 tiles, hi = bf16(w) and
-//     lo = bf16(w - hi) (w - hi is exact in fp32; hi + lo is within 2^-16 |w| of w, so the
-//     contraction carries fp32-like weights and the output rounding keeps the tolerance; one
-//     bf16 weight alone could cost 2^-8 per term), with 16-byte chunks XOR-swizzled by the
-//     row so that both the stores and the transposing loads are conflict-free; the upstream
-//     rows go to a padded tile. ldmatrix gives the A fragments (upstream rows x weight
-//     rows), ldmatrix.trans the B fragments (weight rows x columns: the contraction axis is the
-//     weight's row axis, which the packed codes do not pair), and mma.sync m16n8k16 (bf16 in,
-//     fp32 accumulate) does the contraction, two MMAs (hi, lo) per fragment into one
-//     accumulator; warp w owns columns 32w .. 32w+31. Two buffers,
-//     one barrier per step; the codes, scales and upstream values of the next two steps are in
-//     flight while the current step multiplies. Row splits meet in bwd_x_reduce_kernel as above.
+//   * bwd_x_mma_kernel (2 <= M, K a multiple of 128, N a multiple of 8, 16-byte aligned codes
+//     and dy, 4-byte aligned scales): tensor cores. A CTA owns 128 columns (four scale groups),
+//     a slice of rows and 16 upstream rows. Per step of 32 weight rows each thread unpacks one
+//     32-column group of one row (one 16-byte code load) into a bf16 tile of exact integer
+//     codes in shared memory, 16-byte chunks XOR-swizzled by the row so that both the stores
+//     and the transposing loads are conflict-free, and stores the row's scale; the upstream
+//     rows go to a padded tile. Warp w owns columns 32w .. 32w+31, exactly scale group w: it
+//     loads its A fragments (upstream rows x weight rows) with ldmatrix, multiplies each value
+//     by its weight row's scale in fp32 and splits the product into a bf16 pair hi + lo
+//     (within 2^-16 of it: one bf16 alone could cost 2^-8 per term, too much for the
+//     tolerance once the output is rounded to bf16 as well), loads the B fragments (weight
+//     rows x columns: the contraction runs over the weight's rows, which the packed codes do
+//     not pair) with ldmatrix.trans, and runs two mma.sync m16n8k16 (bf16 in, fp32
+//     accumulate) per fragment. Two buffers, one barrier per step; the codes, scales and
+//     upstream values of the next two steps are in flight while the current step multiplies.
+//     Row splits meet in bwd_x_reduce_kernel as above.
 //   * bwd_x_plain_kernel: any K, one thread per (token, column), rows in order.
 #include "w4_mma.cuh"
 #include "w4_tc.cuh"
@@ -245,36 +245,6 @@ constexpr int kMmaThreads = 128;
 constexpr int kWtPitch = kMmaCols * 2;  // bytes per row of the bf16 weight tile
 constexpr int kDyPitch = 80;            // 32 bf16 + 16 bytes: conflict-free ldmatrix rows
 
-// Eight nibbles of one code word -> the fp32 weights fl32(q * s) of columns 8t .. 8t+7 as two
-// bf16 words per pair: hi = bf16(w), lo = bf16(w - hi), both packed in column order. Per column
-// pair: the nibble (xor 8) in the low byte of the fp32 2^23 (PRMT), one exact fp32x2 subtract of
-// 2^23 + 8 leaves q, one fp32x2 multiply by the scale rounds once; hi is widened back (PRMT /
-// LOP3) and the remainder w - hi (exact) is rounded to bf16.
-__device__ __forceinline__ void dequant_word_split(uint32_t w, uint64_t scale2, uint4 &hi, uint4 &lo) {
-  const uint32_t el = lop3_and_xor(w, 0x0F0F0F0Fu, 0x08080808u);       // even columns, nibble ^ 8
-  const uint32_t od = lop3_and_xor(w >> 4, 0x0F0F0F0Fu, 0x08080808u);  // odd columns
-  const uint64_t nb2 = neg_bias_pair(8u);
-  uint32_t h[4], l[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t fe = prmt(el, 0x00004B00u, 0x5440u | i);
-    const uint32_t fo = prmt(od, 0x00004B00u, 0x5440u | i);
-    uint64_t v = (static_cast<uint64_t>(fo) << 32) | fe;
-    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(nb2));
-    asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(scale2));
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
-        : "=r"(h[i])
-        : "f"(__uint_as_float(static_cast<uint32_t>(v >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(v))));
-    const uint64_t hw = (static_cast<uint64_t>(h[i] & 0xFFFF0000u) << 32) | prmt(h[i], 0u, 0x1044u);
-    asm("sub.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(hw));
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
-        : "=r"(l[i])
-        : "f"(__uint_as_float(static_cast<uint32_t>(v >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(v))));
-  }
-  hi = make_uint4(h[0], h[1], h[2], h[3]);
-  lo = make_uint4(l[0], l[1], l[2], l[3]);
-}
-
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&d)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
@@ -288,12 +258,29 @@ __device__ __forceinline__ void mma_acc(float (&d)[4], const uint32_t (&a)[4], u
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Upstream values of one A-fragment register (two bf16, weight rows n, n + 1) times the two
+// rows' scales, as a pair of bf16x2 registers hi + lo: hi = bf16(fl32(dy * s)), lo = bf16 of
+// the (exact) remainder, so hi + lo is within 2^-16 of the fp32 product.
+__device__ __forceinline__ void scale_split(uint32_t x2, uint64_t s2, uint32_t &hi, uint32_t &lo) {
+  uint64_t v = (static_cast<uint64_t>(x2 & 0xFFFF0000u) << 32) | (x2 << 16);
+  asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(s2));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+      : "=r"(hi)
+      : "f"(__uint_as_float(static_cast<uint32_t>(v >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(v))));
+  const uint64_t hw = (static_cast<uint64_t>(hi & 0xFFFF0000u) << 32) | (hi << 16);
+  asm("sub.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(hw));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+      : "=r"(lo)
+      : "f"(__uint_as_float(static_cast<uint32_t>(v >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(v))));
+}
+
 __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloat16 *__restrict__ dy,
                                                                 const uint8_t *__restrict__ codes,
                                                                 const float *__restrict__ scales, float *part,
                                                                 void *dx, int dx_dtype, int64_t M, int64_t N,
                                                                 int64_t K, int64_t rows_per_split, int splits) {
-  __shared__ __align__(128) uint8_t wt[2][2][kMmaRows * kWtPitch];  // [buffer][hi, lo]
+  __shared__ __align__(128) uint8_t wq[2][kMmaRows * kWtPitch];  // exact codes as bf16 [row][128 columns]
+  __shared__ __align__(16) float wsc[2][4][kMmaRows];             // the step's scales [group][row]
   __shared__ __align__(128) uint8_t dys[2][kMmaTok * kDyPitch];
   const int tid = static_cast<int>(threadIdx.x), warp = tid >> 5, lane = tid & 31;
   const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kMmaCols;
@@ -302,7 +289,7 @@ __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloa
   const int64_t n_begin = static_cast<int64_t>(split) * rows_per_split;
   const int64_t n_end = (n_begin + rows_per_split < N) ? n_begin + rows_per_split : N;
   const int64_t P = K / 2, G = K / 32;
-  // dequant role: row r of the step, the 32 columns of group q of the tile (four code words,
+  // unpack role: row r of the step, the 32 columns of group q of the tile (four code words,
   // one 16-byte load, one scale)
   const int r = tid >> 2, q = tid & 3;
   const uint4 *cw_base = reinterpret_cast<const uint4 *>(codes + k0 / 2) + q;
@@ -326,19 +313,21 @@ __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloa
     st.dv = (dy_row && n0 + q8 < n_end) ? __ldg(reinterpret_cast<const uint4 *>(dy_base + n0))
                                         : make_uint4(0u, 0u, 0u, 0u);
   };
+  // The codes go to the tile as exact integers (one LOP3 and one bf16x2 FMA per column pair);
+  // each 16-byte chunk holds its eight columns in the order 0 4 1 5 2 6 3 7, which the output
+  // indexing undoes. The scale stays fp32 and multiplies the upstream values instead.
   auto put = [&](const Step &st, int buf) {
-    const uint64_t s2 = (static_cast<uint64_t>(__float_as_uint(st.sc)) << 32) | __float_as_uint(st.sc);
     const uint32_t words[4] = {st.cw.x, st.cw.y, st.cw.z, st.cw.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       // the four lanes of a row start at different chunks: fewer bank conflicts on the stores
       const int jj = (j + q) & 3;
-      uint4 vh, vl;
-      dequant_word_split(words[jj], s2, vh, vl);
+      uint32_t a[4];
+      unpack_signed(words[jj], a);
       const int off = r * kWtPitch + (((4 * q + jj) ^ (r & 7)) << 4);
-      *reinterpret_cast<uint4 *>(&wt[buf][0][off]) = vh;
-      *reinterpret_cast<uint4 *>(&wt[buf][1][off]) = vl;
+      *reinterpret_cast<uint4 *>(&wq[buf][off]) = make_uint4(a[0], a[1], a[2], a[3]);
     }
+    wsc[buf][q][r] = st.sc;
     if (tid < 64) *reinterpret_cast<uint4 *>(&dys[buf][tok * kDyPitch + (tid & 3) * 16]) = st.dv;
   };
 
@@ -350,32 +339,40 @@ __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloa
   // B (weight rows x columns, transposed on load): matrix i: rows (l & 7) + 8 (i & 1) of the
   // half, 16-byte chunk 4 warp + pair + (i >> 1)
   const int b_row = lr + 8 * (li & 1);
+  const int g = lane >> 2, t = lane & 3;
 
   float acc[4][4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
 
   const int steps = n_end > n_begin ? static_cast<int>((n_end - n_begin + kMmaRows - 1) / kMmaRows) : 0;
+  // warp w owns columns 32w .. 32w+31: exactly scale group w of the tile
   auto multiply = [&](int buf) {
-    const uint32_t wbase = smem_u32(&wt[buf][0][0]);
+    const uint32_t wbase = smem_u32(&wq[buf][0]);
     const uint32_t dbase = smem_u32(&dys[buf][0]);
-    constexpr uint32_t kLoTile = kMmaRows * kWtPitch;  // lo tile follows the hi tile
+    const float *sw = &wsc[buf][warp][0];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t a[4];
       ldsm_x4(dbase + a_off + 32u * h, a);
+      // the rows of this lane's A registers: 16h + 2t (+1) for a0 / a1, 16h + 2t + 8 (+1) for a2 / a3
+      const uint64_t s01 = *reinterpret_cast<const uint64_t *>(sw + 16 * h + 2 * t);
+      const uint64_t s89 = *reinterpret_cast<const uint64_t *>(sw + 16 * h + 2 * t + 8);
+      uint32_t ah[4], al[4];
+      scale_split(a[0], s01, ah[0], al[0]);
+      scale_split(a[1], s01, ah[1], al[1]);
+      scale_split(a[2], s89, ah[2], al[2]);
+      scale_split(a[3], s89, ah[3], al[3]);
 #pragma unroll
       for (int pr = 0; pr < 2; ++pr) {
         const int row = 16 * h + b_row;
         const int chunk = 4 * warp + 2 * pr + (li >> 1);
-        const uint32_t boff = wbase + static_cast<uint32_t>(row * kWtPitch + ((chunk ^ (row & 7)) << 4));
-        uint32_t b[4], bl[4];
-        ldsm_x4_trans(boff, b);
-        ldsm_x4_trans(boff + kLoTile, bl);
-        mma_acc(acc[2 * pr], a, b[0], b[1]);
-        mma_acc(acc[2 * pr + 1], a, b[2], b[3]);
-        mma_acc(acc[2 * pr], a, bl[0], bl[1]);
-        mma_acc(acc[2 * pr + 1], a, bl[2], bl[3]);
+        uint32_t b[4];
+        ldsm_x4_trans(wbase + static_cast<uint32_t>(row * kWtPitch + ((chunk ^ (row & 7)) << 4)), b);
+        mma_acc(acc[2 * pr], ah, b[0], b[1]);
+        mma_acc(acc[2 * pr], al, b[0], b[1]);
+        mma_acc(acc[2 * pr + 1], ah, b[2], b[3]);
+        mma_acc(acc[2 * pr + 1], al, b[2], b[3]);
       }
     }
   };
@@ -398,11 +395,11 @@ __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloa
     if (it + 2 < steps) put(sa, 0);
   }
 
-  // acc[j]: upstream rows g, g + 8 x columns 32 warp + 8 j + 2 t (+1)
-  const int g = lane >> 2, t = lane & 3;
+  // acc[j]: upstream rows g, g + 8 x tile positions 2t, 2t + 1 of column chunk 4 warp + j,
+  // which hold columns t and t + 4 of the chunk
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int64_t kk = k0 + 32 * warp + 8 * j + 2 * t;
+    const int64_t kk = k0 + 32 * warp + 8 * j + t;
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
       const int64_t m = m0 + g + 8 * hf;
@@ -410,11 +407,11 @@ __global__ void __launch_bounds__(kMmaThreads) bwd_x_mma_kernel(const __nv_bfloa
       const float v0 = acc[j][2 * hf], v1 = acc[j][2 * hf + 1];
       if (splits == 1) {
         store_out(dx, dx_dtype, m * K + kk, v0);
-        store_out(dx, dx_dtype, m * K + kk + 1, v1);
+        store_out(dx, dx_dtype, m * K + kk + 4, v1);
       } else {
         float *dst = part + (static_cast<int64_t>(split) * M + m) * K + kk;
         dst[0] = v0;
-        dst[1] = v1;
+        dst[4] = v1;
       }
     }
   }
