@@ -657,6 +657,27 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
         return ([lambda r=r: step(r) for r in range(ROTATE)],
                 lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
 
+    def lora_merge(r):
+        # merge a rank-r adapter into the (14336, 4096) projection and re-quantize it (an offline
+        # call): codes and scales read and written (separate output copies, so that every call
+        # merges the same weight), the two factors read once
+        def make():
+            N, K = workloads.BATCHED_SHAPE
+            c = workloads.decode_case(N, K, M=1, config=3)
+            codes, scales = w4.quantize_rtn(torch.from_numpy(c["W"]).to(dev))
+            copies = [(codes.clone(), scales.clone()) for _ in range(ROTATE)]
+            g = torch.Generator(device="cpu").manual_seed(11)
+            bt = (torch.randn(N, r, generator=g) * 0.01).to(dev)
+            at = (torch.randn(r, K, generator=g) * 0.01).to(dev)
+            outs = [(torch.empty_like(codes), torch.empty_like(scales)) for _ in range(ROTATE)]
+            st = torch.zeros(1, dtype=torch.int32, device=dev)
+            nb = 2 * payload(N, K) + 4 * r * (N + K)
+            return ([lambda c=c, s=s, o=o: w4.lora_merge(c, s, K, bt, at, 2.0, out=o, status=st)
+                     for (c, s), o in zip(copies, outs)],
+                    lambda us: {"us": us, "gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak,
+                                "rank": r})
+        return make
+
     def backward_x(M):
         # input gradient dx = dy . dequant(W) of the (14336, 4096) projection
         def make():
@@ -675,7 +696,7 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
         return make
 
     w = {"dequant_4096x4095_bf16": dequant_odd, "quantize_14336x4096": quantize, "q4_0_decode_M1_step": q4_0_decode,
-         "channel_decode_M1_step": channel_decode,
+         "channel_decode_M1_step": channel_decode, "lora_merge_r16_14336x4096": lora_merge(16),
          "backward_x_M1_14336x4096": backward_x(1), "backward_x_M16_14336x4096": backward_x(16)}
     for M in workloads.BATCHED_M:
         w[f"batched_M{M}_14336x4096"] = batched(M)

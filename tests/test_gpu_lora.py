@@ -37,7 +37,7 @@ def lora_case(N, K, r, seed):
 
 
 @pytest.mark.parametrize("NKr", [(1, 1, 1), (3, 7, 2), (37, 333, 3), (64, 4096, 16), (300, 1000, 8), (5, 96, 64),
-                                 (9, 40, 0)])
+                                 (9, 40, 0), (33, 129, 17), (70, 520, 40), (256, 1024, 16), (31, 127, 1)])
 def test_lora_merge_bit_exact(w4, NKr):
     N, K, r = NKr
     codes, s, b, a = lora_case(N, K, r, N + K + r)
@@ -50,6 +50,22 @@ def test_lora_merge_bit_exact(w4, NKr):
     # in place
     w4.lora_merge(dc, ds, K, dev(b) if r else None, dev(a) if r else None, c, out=(dc, ds))
     assert torch.equal(dc, co) and torch.equal(ds, so)
+
+
+def test_lora_merge_ties_and_near_ties(w4):
+    # merged values on and 2^-22 beside half-integers of the new scale, with scales whose
+    # reciprocal is exact in fp32 (1, 2^-20) and inexact (3, 3/8, 1/3, 5, 7): the codes round
+    # half to even exactly as the oracle's division does
+    from test_lora_oracle import lora_tie_case
+    scales = [1.0, 3.0, 0.375, float(np.float32(1 / 3)), 5.0, 1.0, 2.0**-20, 7.0]
+    codes, s, b, a, q, d = lora_tie_case(scales)
+    q2, s2 = O.lora_merge(codes, s, 64, b, a, 1.0)
+    co, so = w4.lora_merge(dev(codes), dev(s), 64, dev(b), dev(a), 1.0)
+    assert np.array_equal(co.cpu().numpy(), O.pack_nibbles(q2))
+    assert np.array_equal(so.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+    unit = [i for i, v in enumerate(scales) if v == 1.0]
+    expect = np.vectorize(lambda v: round(v))(q + d)[unit]
+    assert np.array_equal(q2[unit].astype(np.int64), expect)
 
 
 def test_lora_merge_worked_example_on_device(w4):

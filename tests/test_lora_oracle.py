@@ -1,8 +1,9 @@
 """Pins of the LoRA-merge oracle (Keras page, Dense's merged-kernel helper: dequantize,
 add (alpha / rank) * A . B, re-quantize, pack): hand-worked merges with exact arithmetic
 (tests/golden/lora_merge_worked_example.txt), the zero update reducing to re-quantizing the
-dequantized weight (two pinned functions), a rank-one update equal to its closed form, and
-planted mistakes that a pin must catch."""
+dequantized weight (two pinned functions), a rank-one update equal to its closed form,
+merged values on and 2^-22 beside half-integers re-quantizing half to even, and planted
+mistakes that a pin must catch."""
 
 import numpy as np
 import pytest
@@ -55,7 +56,47 @@ def pin_lora_rank_one_closed_form(o):
     assert np.array_equal(q, q3) and np.array_equal(s2, s3)
 
 
-PINS = [pin_lora_worked, pin_lora_zero_update, pin_lora_rank_one_closed_form]
+# offsets of the merged value from its code q: exact half-integer ties and values 2^-22 to
+# either side of one (exact in fp32 while |q + d| < 4), and 0
+TIE_OFFSETS = (0.5, -0.5, 0.5 + 2.0**-22, 0.5 - 2.0**-22, -0.5 + 2.0**-22, -0.5 - 2.0**-22, 1.5, -1.5, 0.0)
+
+
+def lora_tie_case(row_scales):
+    """A rank-one merge (c = 1) whose merged values sit on or 2^-22 beside half-integers of
+    the row's scale: K = 64 (two groups); column 0 of each group keeps code 7 and offset 0, so
+    the group's amax is 7 s and its new scale s again; the other columns take codes in
+    -3 .. 2 and an offset d from TIE_OFFSETS through b[n] = s[n], a[0, k] = d. Returns
+    (codes, scales, b, a, q, d) with q and d the [N, 64] codes and offsets."""
+    N, K = len(row_scales), 64
+    q = np.zeros((N, K), np.int64)
+    d = np.zeros((N, K))
+    qs = (-3, -2, -1, 0, 1, 2)
+    for n in range(N):
+        for k in range(K):
+            if k % 32 == 0:
+                q[n, k] = 7
+            else:
+                q[n, k] = qs[(5 * k + n) % len(qs)]
+                d[n, k] = TIE_OFFSETS[k % len(TIE_OFFSETS)]
+    # one offset per column: rows share a (rank one), so every row takes column k's offset
+    d[:] = d[0]
+    s = np.repeat(np.asarray(row_scales, np.float32).reshape(N, 1), 2, axis=1)
+    b = np.asarray(row_scales, np.float32).reshape(N, 1)
+    a = d[0:1].astype(np.float32)
+    return O.pack_nibbles(q), s, b, a, q, d
+
+
+def pin_lora_half_even_ties(o):
+    # unit scales: every step is exact, so the new codes are round-half-even(q + d) and the
+    # scales stay 1
+    codes, s, b, a, q, d = lora_tie_case([1.0, 1.0, 1.0])
+    q2, s2 = o.lora_merge(codes, s, 64, b, a, 1.0)
+    expect = np.vectorize(lambda v: round(v))(q + d)  # Python's round() is half to even
+    assert np.array_equal(q2.astype(np.int64), expect)
+    assert np.array_equal(s2, np.ones_like(s2))
+
+
+PINS = [pin_lora_worked, pin_lora_zero_update, pin_lora_rank_one_closed_form, pin_lora_half_even_ties]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -92,3 +133,20 @@ def test_mutant_lora_alpha_ignored():
 
 def test_mutant_lora_rank_rows_swapped():
     _fails(lambda *args: _merge(*args, transpose=True), pin_lora_worked)
+
+
+def _merge_half_away(codes, scales, K, b, a, c):
+    w = O.dequantize(codes, scales, K, "f32")
+    t = (np.asarray(b, np.float32) @ np.asarray(a, np.float32)).astype(np.float32)
+    m = (w + (np.float32(c) * t).astype(np.float32)).astype(np.float32)
+    g = m.reshape(m.shape[0], -1, 32)
+    s2 = np.maximum((np.abs(g).max(axis=2) / np.float32(7)).astype(np.float32), np.finfo(np.float32).tiny)
+    x = (g / s2[:, :, None]).astype(np.float32)
+    qq = np.clip(np.sign(x) * np.floor(np.abs(x) + 0.5), -7, 7).astype(np.int8)
+    return qq.reshape(m.shape), s2.astype(np.float32)
+
+
+def test_mutant_lora_ties_away_from_zero():
+    codes, s, b, a = lora_tie_case([1.0])[:4]
+    assert np.array_equal(_merge_half_away(codes, s, 64, b, a, 1.0)[1], np.ones((1, 2), np.float32))
+    _fails(_merge_half_away, pin_lora_half_even_ties)

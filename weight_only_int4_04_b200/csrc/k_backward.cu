@@ -260,7 +260,9 @@ __device__ __forceinline__ void mma_acc(float (&d)[4], const uint32_t (&a)[4], u
 
 // Upstream values of one A-fragment register (two bf16, weight rows n, n + 1) times the two
 // rows' scales, as a pair of bf16x2 registers hi + lo: hi = bf16(fl32(dy * s)), lo = bf16 of
-// the (exact) remainder, so hi + lo is within 2^-16 of the fp32 product.
+// the (exact) remainder, so hi + lo is within 2^-16 of the fp32 product. (ptxas may fuse the
+// packed multiply and subtract into one fma; lo is then the remainder of the exact product,
+// which only tightens the bound.)
 __device__ __forceinline__ void scale_split(uint32_t x2, uint64_t s2, uint32_t &hi, uint32_t &lo) {
   uint64_t v = (static_cast<uint64_t>(x2 & 0xFFFF0000u) << 32) | (x2 << 16);
   asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(v) : "l"(s2));
