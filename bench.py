@@ -672,9 +672,14 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
             outs = [(torch.empty_like(codes), torch.empty_like(scales)) for _ in range(ROTATE)]
             st = torch.zeros(1, dtype=torch.int32, device=dev)
             nb = 2 * payload(N, K) + 4 * r * (N + K)
+            # the rank sum is r separately rounded products and r sums per weight in scalar fp32,
+            # so the call is bound by fp32 issue: 148 SMs x 128 lanes x the 1965 MHz maximum clock
+            ops = 2 * N * K * r
+            fp32_peak = 148 * 128 * 1.965e9
             return ([lambda c=c, s=s, o=o: w4.lora_merge(c, s, K, bt, at, 2.0, out=o, status=st)
                      for (c, s), o in zip(copies, outs)],
                     lambda us: {"us": us, "gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak,
+                                "fp32_tops": ops / us / 1e6, "frac_fp32": ops / (us * 1e-6) / fp32_peak,
                                 "rank": r})
         return make
 

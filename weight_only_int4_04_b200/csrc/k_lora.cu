@@ -14,7 +14,7 @@
 //     steps, transposed) are double-buffered with cp.async: the next step's copies are in
 //     flight while the current one computes. A thread owns 4 rows x 4 consecutive columns
 //     (the 8 lanes of a quarter warp cover one 32-column group of one row); its code bytes
-//     and scales are loaded into registers when the tile starts and used by the epilogue,
+//     and scales are loaded into registers one tile ahead and used by the epilogue,
 //     which dequantizes, adds c * t, reduces each group's amax over its 8 lanes by shuffles
 //     and writes codes and scale. A code byte belongs to one group and a tile to one CTA, so
 //     the output may overwrite the input.
@@ -31,7 +31,7 @@ constexpr int kLoraRows = 32;     // tile rows: 8 warps x 4 rows
 constexpr int kLoraCols = 128;    // tile columns: 4 groups of 32
 constexpr int kLoraChunk = 32;    // rank steps staged at a time
 constexpr int kLoraBPitch = 36;   // b slice row pitch (floats): 16-B aligned rows for the float4 reads
-constexpr int kLoraCtasPerSm = 3;
+constexpr int kLoraCtasPerSm = 2;
 
 struct LoraSmem {
   float a[2][kLoraChunk][kLoraCols];    // a[j0 + jj][k0 + cc]
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kLoraThreads, kLoraCtasPerSm)
   const int ncols = c0 >= K ? 0 : (K - c0 >= 4 ? 4 : static_cast<int>(K - c0));
   const int64_t g = c0 / 32;
   const int64_t jb = c0 / 2;  // code bytes jb (columns c0, c0+1) and jb+1
-  const bool two_bytes = jb + 1 < P;
+  const bool two_bytes = jb + 1 < P;  // false: columns c0 + 2, c0 + 3 are past K
   const int nch = static_cast<int>((r + kLoraChunk - 1) / kLoraChunk);
   int a_tag0 = -1, a_tag1 = -1;  // the chunk each a buffer holds; block-uniform
 
@@ -135,32 +135,36 @@ __global__ void __launch_bounds__(kLoraThreads, kLoraCtasPerSm)
     }
     cp_async_commit();
   };
-  // the thread's code words (two bytes per row) and scales of row tile it
-  auto load_tile = [&](int64_t it, uint32_t (&word)[4], float (&sc)[4]) {
+  // the thread's two code bytes per row and scales of row tile it. The addresses are clamped
+  // into the arrays and the loads are unconditional, so nothing consumes a loaded value before
+  // the epilogue of the tile (which discards rows and columns outside the weight): the loads
+  // of the next tile stay in flight through this tile's rank loop.
+  const int64_t jb_lo = jb < P - 1 ? jb : P - 1;
+  const int64_t jb_hi = jb + 1 < P - 1 ? jb + 1 : P - 1;
+  const int64_t g_in = g < G - 1 ? g : G - 1;
+  auto load_tile = [&](int64_t it, uint32_t (&lo)[4], uint32_t (&hi)[4], float (&sc)[4]) {
     const int64_t n0 = (rt0 + it * walkers) * kLoraRows;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int64_t n = n0 + rl + i;
-      word[i] = 0u;
-      sc[i] = 0.0f;
-      if (n < N && ncols > 0) {
-        const uint8_t *crow = codes + n * P;
-        word[i] = crow[jb] | (two_bytes ? static_cast<uint32_t>(crow[jb + 1]) << 8 : 0u);
-        sc[i] = scales[n * G + g];
-      }
+      const int64_t n = n0 + rl + i < N ? n0 + rl + i : N - 1;
+      const uint8_t *crow = codes + n * P;
+      lo[i] = crow[jb_lo];
+      hi[i] = crow[jb_hi];
+      sc[i] = scales[n * G + g_in];
     }
   };
 
+  if (my_tiles <= 0) return;
   float chk = 0.0f;  // becomes NaN once any merged value is not finite
-  uint32_t word[4];
+  uint32_t lo[4], hi[4];
   float sc[4];
-  load_tile(0, word, sc);
+  load_tile(0, lo, hi, sc);
   if (nch > 0) issue(0, 0, 0);
   int buf = 0;
   for (int64_t it = 0; it < my_tiles; ++it) {
-    uint32_t word_next[4] = {0u, 0u, 0u, 0u};
-    float sc_next[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (it + 1 < my_tiles) load_tile(it + 1, word_next, sc_next);
+    uint32_t lo_next[4], hi_next[4];
+    float sc_next[4];
+    load_tile(it + 1 < my_tiles ? it + 1 : it, lo_next, hi_next, sc_next);
     float t[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -194,7 +198,7 @@ __global__ void __launch_bounds__(kLoraThreads, kLoraCtasPerSm)
       am[i] = 0.0f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float wv = __fadd_rn(__fmul_rn(lora_code(word[i], e), sc[i]), __fmul_rn(c, t[i][e]));
+        const float wv = __fadd_rn(__fmul_rn(lora_code(lo[i] | (hi[i] << 8), e), sc[i]), __fmul_rn(c, t[i][e]));
         const bool in = e < ncols && n0 + rl + i < N;
         t[i][e] = in ? wv : 0.0f;  // t now holds w'
         chk = __fmaf_rn(t[i][e], 0.0f, chk);
@@ -249,7 +253,8 @@ __global__ void __launch_bounds__(kLoraThreads, kLoraCtasPerSm)
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      word[i] = word_next[i];
+      lo[i] = lo_next[i];
+      hi[i] = hi_next[i];
       sc[i] = sc_next[i];
     }
   }
