@@ -64,8 +64,16 @@ __device__ __forceinline__ void lora_rank_step(const float *a_row, const float *
 }
 
 // signed value of nibble e of a code word, as an exact fp32: (u ^ 8) - 8 through the 2^23 bias
+// (the bias's bits and the nibble's are disjoint, so one xor sets both)
 __device__ __forceinline__ float lora_code(uint32_t word, int e) {
-  return __fsub_rn(__uint_as_float(0x4B000000u | (((word >> (4 * e)) & 15u) ^ 8u)), 8388616.0f);
+  return __fsub_rn(__uint_as_float(((word >> (4 * e)) & 15u) ^ 0x4B000008u), 8388616.0f);
+}
+
+// max that returns NaN when either input is NaN, so a group's amax carries a NaN merged value
+__device__ __forceinline__ float lora_max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
 // code nibble of round-half-even(fl32(w / s2)), where |w / s2| < 8 (|w| <= amax, s2 >= amax / 7).
@@ -77,8 +85,7 @@ __device__ __forceinline__ float lora_code(uint32_t word, int e) {
 __device__ __forceinline__ uint32_t lora_rtn_nibble(float w, float y, bool &near) {
   const float x = __fmul_rn(w, y);
   const float xm = __fadd_rn(x, 12582912.0f);
-  const float d = fabsf(__fsub_rn(x, __fsub_rn(xm, 12582912.0f)));
-  near |= fabsf(__fsub_rn(d, 0.5f)) < 0x1p-18f;
+  near |= fabsf(__fsub_rn(x, __fsub_rn(xm, 12582912.0f))) > 0.5f - 0x1p-18f;
   return __float_as_uint(xm) & 15u;
 }
 
@@ -155,7 +162,7 @@ __global__ void __launch_bounds__(kLoraThreads, kLoraCtasPerSm)
   };
 
   if (my_tiles <= 0) return;
-  float chk = 0.0f;  // becomes NaN once any merged value is not finite
+  bool bad = false;  // a non-finite merged value was seen
   uint32_t lo[4], hi[4];
   float sc[4];
   load_tile(0, lo, hi, sc);
@@ -190,31 +197,34 @@ __global__ void __launch_bounds__(kLoraThreads, kLoraCtasPerSm)
       __syncthreads();  // buffers buf are free for the step after next
       buf ^= 1;
     }
-    // epilogue: w' = fl32(fl32(q * s) + fl32(c * t)), then RTN over each row's group
+    // epilogue: w' = fl32(fl32(q * s) + fl32(c * t)), then RTN over each row's group.
+    // Columns past K have zero codes (masked here) and t = 0 (zero-filled a), so w' = 0 there;
+    // rows past N repeat row N - 1 (clamped loads) and are never stored.
     const int64_t n0 = (rt0 + it * walkers) * kLoraRows;
+    const uint32_t colmask = ncols >= 4 ? 0xFFFFu : ((1u << (4 * ncols)) - 1u);
     float am[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
+      const uint32_t word = (lo[i] | (hi[i] << 8)) & colmask;
       am[i] = 0.0f;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float wv = __fadd_rn(__fmul_rn(lora_code(lo[i] | (hi[i] << 8), e), sc[i]), __fmul_rn(c, t[i][e]));
-        const bool in = e < ncols && n0 + rl + i < N;
-        t[i][e] = in ? wv : 0.0f;  // t now holds w'
-        chk = __fmaf_rn(t[i][e], 0.0f, chk);
-        am[i] = fmaxf(am[i], fabsf(t[i][e]));
+        t[i][e] = __fadd_rn(__fmul_rn(lora_code(word, e), sc[i]), __fmul_rn(c, t[i][e]));  // t now holds w'
+        am[i] = lora_max_nan(am[i], fabsf(t[i][e]));
       }
     }
-    // the 8 lanes of a quarter warp hold one group of each of the 4 rows: reduce the amax,
-    // then lane (sub & 3) of the group forms row (sub & 3)'s scale and reciprocal for all
+    // the 8 lanes of a quarter warp hold one group of each of the 4 rows: reduce the amax
+    // (NaN-propagating, so a non-finite merged value shows in its row's amax), then lane
+    // (sub & 3) of the group forms row (sub & 3)'s scale and reciprocal for all
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      am[i] = fmaxf(am[i], __shfl_xor_sync(0xffffffffu, am[i], 1));
-      am[i] = fmaxf(am[i], __shfl_xor_sync(0xffffffffu, am[i], 2));
-      am[i] = fmaxf(am[i], __shfl_xor_sync(0xffffffffu, am[i], 4));
+      am[i] = lora_max_nan(am[i], __shfl_xor_sync(0xffffffffu, am[i], 1));
+      am[i] = lora_max_nan(am[i], __shfl_xor_sync(0xffffffffu, am[i], 2));
+      am[i] = lora_max_nan(am[i], __shfl_xor_sync(0xffffffffu, am[i], 4));
     }
     const int pick = lane & 3;
     const float mine = pick == 0 ? am[0] : (pick == 1 ? am[1] : (pick == 2 ? am[2] : am[3]));
+    bad |= !(mine <= FLT_MAX);  // a NaN or infinite merged value in the row's group
     const float s2_mine = fmaxf(__fdiv_rn(mine, 7.0f), FLT_MIN);
     const float y_mine = __frcp_rn(s2_mine);
     float s2[4], y[4];
@@ -239,7 +249,6 @@ __global__ void __launch_bounds__(kLoraThreads, kLoraCtasPerSm)
     // columns past K keep a zero pad nibble. The output may alias the input: a lane writes
     // only the two code bytes it read itself, and the group's scale, read by its eight lanes
     // before the shuffles, is written after
-    const uint32_t colmask = ncols >= 4 ? 0xFFFFu : ((1u << (4 * ncols)) - 1u);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int64_t n = n0 + rl + i;
@@ -258,7 +267,7 @@ __global__ void __launch_bounds__(kLoraThreads, kLoraCtasPerSm)
       sc[i] = sc_next[i];
     }
   }
-  if (!(fabsf(chk) <= FLT_MAX)) *status = W4_ERR_NONFINITE;
+  if (bad) *status = W4_ERR_NONFINITE;
 }
 
 }  // namespace
