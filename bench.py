@@ -638,6 +638,29 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
         return ([lambda r=r: step(r) for r in range(ROTATE)],
                 lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak})
 
+    def q4_0_as_group32_decode():
+        # the same Q4_0 decode step after a one-time re-layout of every block copy into the
+        # group-32 format (w4_q4_0_to_group32, outside the timed region): the group-32 decode
+        # GEMV then streams 20 bytes per 32 weights. Throughput is counted in the blocks'
+        # 18 bytes per 32 weights, so that the row compares with q4_0_decode_M1_step;
+        # stream_gbs counts the bytes actually read
+        sets, xs, ys, nb, ns = [], [], [], 0, 0
+        for N, K in workloads.Q4_0_SHAPES:
+            c = workloads.q4_0_case(N + K, 1, N, K, bias=False)
+            blk = torch.from_numpy(c["blocks"]).to(dev)
+            sets.append([w4.Linear(*w4.q4_0_to_group32(blk, K), None, K) for _ in range(ROTATE)])
+            xs.append(bf16(c["x_bits"]))
+            ys.append(torch.empty((1, N), dtype=torch.bfloat16, device=dev))
+            nb += N * (K // 32) * 18
+            ns += payload(N, K)
+
+        def step(r):
+            for j in range(len(xs)):
+                sets[j][r](xs[j], out=ys[j])
+        return ([lambda r=r: step(r) for r in range(ROTATE)],
+                lambda us: {"us": us, "weight_gbs": nb / us / 1e3, "frac_hbm": nb / us / 1e3 / hbm_peak,
+                            "stream_gbs": ns / us / 1e3})
+
     def channel_decode():
         # the headline's decode step on per-channel weights (one fp32 scale per row, read by
         # the decode kernel: 0.5 bytes per weight + 4 per row)
@@ -701,6 +724,7 @@ def detail_workloads(w4, dev, hbm_peak, tc_peak):
         return make
 
     w = {"dequant_4096x4095_bf16": dequant_odd, "quantize_14336x4096": quantize, "q4_0_decode_M1_step": q4_0_decode,
+         "q4_0_as_group32_decode_M1_step": q4_0_as_group32_decode,
          "channel_decode_M1_step": channel_decode, "lora_merge_r16_14336x4096": lora_merge(16),
          "backward_x_M1_14336x4096": backward_x(1), "backward_x_M16_14336x4096": backward_x(16)}
     for M in workloads.BATCHED_M:

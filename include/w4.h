@@ -336,6 +336,26 @@ w4_status w4_linear_q4_0(const void *x, int64_t M, const uint8_t *blocks, int64_
                          const float *bias, void *y, w4_dtype y_dtype, w4_stream_t stream);
 
 /*
+ * w4_q4_0_to_group32 -- re-lay Q4_0 blocks out as this library's packed group-32 format, once
+ * per weight (at load time). MAX page (max/python/max/graph/quantization.py),
+ * QuantizationEncoding.Q4_0: a block is 32 consecutive columns of a row with one scale, and
+ * its value d * (c - 8) is scale * code with
+ *     scales[n][g] = fp32(d[n][g])                 (binary16 widened exactly)
+ *     code of column k = c[n][k] - 8 in [-8, 7]    (a two's-complement nibble; -8 is the
+ *                                                   format-v2 code, accepted by every call)
+ * so w4_linear, w4_dequantize, w4_linear_backward_x ... on (codes, scales) see exactly the
+ * dequantized weights of the blocks: fp32(scale * code) = fp32(d * (c - 8)), both exact.
+ * Any binary16 d is carried over (negative, zero, subnormal; a non-finite d becomes a
+ * non-finite scale, which w4_validate reports).
+ *   blocks  uint8 [N, K/32, 18] (device), K a multiple of 32; not modified.
+ *   codes   uint8 [N, K/2] (device, caller-owned, written); scales float32 [N, K/32]
+ *           (device, caller-owned, written). Neither may overlap the blocks.
+ * Errors: W4_ERR_NULL, W4_ERR_SHAPE (sizes, K not a multiple of 32), W4_ERR_CUDA.
+ */
+w4_status w4_q4_0_to_group32(const uint8_t *blocks, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                             w4_stream_t stream);
+
+/*
  * w4_set_weight_prefetch -- launch policy of the decode linear (process-wide; default 0).
  * The source pages have no counterpart to this call: it only decides when a kernel starts.
  * The M = 1 decode kernel is launched with CUDA programmatic dependent launch: it may begin

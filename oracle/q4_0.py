@@ -115,6 +115,20 @@ def pack(d, c) -> np.ndarray:
     return np.concatenate([dbytes, q], axis=2)
 
 
+def to_group32(blocks, K: int):
+    """The blocks re-laid out as this library's packed group-32 format.
+
+    A Q4_0 block is a group of 32 consecutive columns with one scale: element value
+    ``d * (c - 8)`` is ``s * q`` with ``s = d`` (binary16 widened exactly to fp32) and the
+    signed code ``q = c - 8`` in [-8, 7] (format v2). Returns ``(codes, scales)``: ``codes``
+    uint8 ``[N, K/2]`` as :func:`w4_oracle.pack_nibbles` packs ``q`` (even column in the low
+    nibble, two's complement), ``scales`` float32 ``[N, K/32]``. Every group-32 dequantization
+    of the result equals :func:`dequantize` of the blocks (both products are exact)."""
+    d, c = unpack(blocks, K)
+    q = c.astype(np.int16) - OFFSET
+    return _w4.pack_nibbles(q), d.astype(np.float32)
+
+
 def validate(blocks, K: int) -> str:
     """"OK" when every block scale is finite, else "SCALE" (a reading: the page states no
     rule; a non-finite d turns every element of its block into NaN or infinity)."""

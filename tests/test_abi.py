@@ -167,6 +167,19 @@ def test_lora_host_checks(w4):
     assert L.w4_lora_merge(FAKE, FAKE, 0, 64, FAKE, FAKE, 2, c, FAKE, FAKE, None, None) == 2
 
 
+def test_q4_0_to_group32_host_checks(w4):
+    L = w4.lib
+    FAKE = ctypes.c_void_p(0x1000)
+    assert L.w4_q4_0_to_group32(None, 4, 64, FAKE, FAKE, None) == 1
+    assert L.w4_q4_0_to_group32(FAKE, 4, 64, None, FAKE, None) == 1
+    assert L.w4_q4_0_to_group32(FAKE, 4, 64, FAKE, None, None) == 1
+    assert L.w4_q4_0_to_group32(FAKE, 4, 48, FAKE, FAKE, None) == 2  # K not a multiple of 32
+    assert L.w4_q4_0_to_group32(FAKE, 0, 64, FAKE, FAKE, None) == 2
+    import torch
+    with pytest.raises(ValueError):  # CPU tensors: no fallback
+        w4.q4_0_to_group32(torch.zeros((4, 2, 18), dtype=torch.uint8), 64)
+
+
 def test_new_bindings_validate_arguments(w4):
     import torch
     f32 = torch.zeros((4, 64), dtype=torch.float32)

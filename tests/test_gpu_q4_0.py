@@ -155,3 +155,39 @@ def test_q4_0_group32_reduction_on_device(w4):
     y2 = w4.linear(x_dev(xb), dev(codes), dev(d), K, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
     check(y1, yr, bound, "q4_0")
     check(y2, yr, bound, "group-32")
+
+
+@pytest.mark.parametrize("NK", [(1, 32), (3, 96), (17, 256), (64, 1056), (129, 4096)])
+def test_q4_0_to_group32_bit_exact(w4, NK):
+    # the re-laid-out codes and scales equal the oracle's, byte for byte (binary16 edge scales
+    # included), with the codes written through the 16-byte path and through the byte path
+    # (an output that starts one byte past a 16-byte boundary)
+    N, K = NK
+    blocks = special_blocks(N, K)
+    codes_ref, scales_ref = Q.to_group32(blocks, K)
+    db = dev(blocks)
+    codes, scales = w4.q4_0_to_group32(db, K)
+    assert np.array_equal(codes.cpu().numpy(), codes_ref), NK
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), scales_ref.view(np.uint32)), NK
+    buf = torch.zeros(N * (K // 2) + 1, dtype=torch.uint8, device="cuda")
+    c2 = buf[1:]
+    s2 = torch.empty(N * (K // 32), dtype=torch.float32, device="cuda")
+    w4.q4_0_to_group32(db, K, out=(c2, s2))
+    assert np.array_equal(c2.cpu().numpy().reshape(N, K // 2), codes_ref), NK
+    assert int(buf[0]) == 0
+
+
+@pytest.mark.parametrize("case", [(1, 300, 4096), (1, 4096, 4096), (1, 17, 512), (16, 100, 1024), (33, 64, 2048)],
+                         ids=lambda c: f"M{c[0]}_N{c[1]}_K{c[2]}")
+def test_q4_0_group32_linear(w4, case):
+    # the group-32 linear on the re-laid-out weight meets the Q4_0 oracle's tolerance
+    M, N, K = case
+    c = workloads.q4_0_case(M * 1000003 + N * 101 + K + 5, M, N, K)
+    yr, bound = Q.linear(c["x"], c["blocks"], K, c["bias"])
+    codes, scales = w4.q4_0_to_group32(dev(c["blocks"]), K)
+    y = w4.linear(x_dev(c["x_bits"]), codes, scales, K, bias=dev(c["bias"]), out_dtype=torch.float32)
+    check(y.cpu().numpy().astype(np.float64), yr, bound, (M, N, K, "group-32"))
+    layer = w4.Linear(codes, scales, dev(c["bias"]), K) if M <= 16 else None
+    if layer is not None:
+        check(layer(x_dev(c["x_bits"]), out_dtype=torch.float32).cpu().numpy().astype(np.float64), yr, bound,
+              (M, N, K, "Linear"))

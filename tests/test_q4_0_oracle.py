@@ -104,6 +104,26 @@ def pin_q4_0_group32_reduction(q):
     assert np.array_equal(y1, y2) and np.array_equal(b1, b2)
 
 
+def pin_q4_0_to_group32(q):
+    # the re-laid-out weight dequantizes (group-32 oracle) to exactly the blocks' weight, for
+    # scales of both signs, signed zero, a binary16 subnormal and the largest binary16 value,
+    # and every code including c = 0 (q = -8)
+    rng = np.random.default_rng(12)
+    N, K = 9, 96
+    d = (rng.standard_normal((N, K // 32)) * 0.01).astype(np.float32)
+    d[0, 0], d[1, 1], d[2, 2], d[3, 0] = 0.0, -0.0, 2.0**-24, -65504.0
+    c = rng.integers(0, 16, size=(N, K))
+    c[0, :16] = np.arange(16)
+    blocks = q.pack(d, c)
+    codes, scales = q.to_group32(blocks, K)
+    assert codes.dtype == np.uint8 and codes.shape == (N, K // 2)
+    assert scales.dtype == np.float32 and scales.shape == (N, K // 32)
+    assert np.array_equal(O.dequantize(codes, scales, K, "f32"), q.dequantize(blocks, K, "f32"))
+    # by hand: columns 0 and 1 of row 0 hold codes 0 and 1, i.e. q = -8 and -7, nibbles 8 and 9
+    assert codes[0, 0] == 0x98 and codes[0, 7] == 0x76  # columns 14, 15: q = 6, 7
+    assert scales[2, 2] == np.float32(2.0**-24) and scales[3, 0] == np.float32(-65504.0)
+
+
 def pin_q4_0_pack_roundtrip(q):
     blocks = workloads.q4_0_case(5, 1, 7, 96)["blocks"]
     d, c = q.unpack(blocks, 96)
@@ -112,7 +132,7 @@ def pin_q4_0_pack_roundtrip(q):
 
 
 PINS = [pin_q4_0_worked, pin_q4_0_binary16, pin_q4_0_code_bytes, pin_q4_0_one_hot, pin_q4_0_group32_reduction,
-        pin_q4_0_pack_roundtrip]
+        pin_q4_0_to_group32, pin_q4_0_pack_roundtrip]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -199,3 +219,24 @@ def test_mutant_q4_0_scale_rounded_to_bf16(monkeypatch):
         return w
     monkeypatch.setattr(Q, "dequantize", deq_bf16)
     _fails(pin_q4_0_group32_reduction)
+
+
+def test_mutant_q4_0_to_group32_bytes_copied(monkeypatch):
+    # the block's code bytes copied as they are (element j / j + 16 per byte kept), offset applied
+    def copied(blocks, K):
+        b = np.ascontiguousarray(blocks, dtype=np.uint8)
+        d = np.ascontiguousarray(b[:, :, 0:2]).view("<f2")[:, :, 0].astype(np.float32)
+        return (b[:, :, 2:] ^ np.uint8(0x88)).reshape(b.shape[0], K // 2), d
+    monkeypatch.setattr(Q, "to_group32", copied)
+    _fails(pin_q4_0_to_group32)
+
+
+def test_mutant_q4_0_to_group32_unsigned(monkeypatch):
+    # codes c stored without the offset
+    orig_unpack = Q.unpack
+
+    def unsigned(blocks, K):
+        d, c = orig_unpack(blocks, K)
+        return O.pack_nibbles(c.astype(np.int16)), d
+    monkeypatch.setattr(Q, "to_group32", unsigned)
+    _fails(pin_q4_0_to_group32)

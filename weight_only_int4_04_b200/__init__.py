@@ -34,7 +34,7 @@ EXPORTS = (
     "w4_set_weight_prefetch", "w4_device_error", "w4_last_cuda_error", "w4_status_string", "w4_version",
     "w4_dequantize_q4_0", "w4_linear_q4_0", "w4_linear_backward_x_workspace_bytes", "w4_linear_backward_x",
     "w4_quantize_rtn_channel", "w4_expand_channel_scales", "w4_lora_merge", "w4_selftest_wait_timeout",
-    "w4_last_linear_kernel", "w4_linear_channel_workspace_bytes", "w4_linear_channel",
+    "w4_last_linear_kernel", "w4_linear_channel_workspace_bytes", "w4_linear_channel", "w4_q4_0_to_group32",
 )
 
 _vp, _i64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -56,6 +56,7 @@ _SIGS = {
     "w4_status_string": [_i32],
     "w4_version": [],
     "w4_dequantize_q4_0": [_vp, _i64, _i64, _i32, _vp, _vp],
+    "w4_q4_0_to_group32": [_vp, _i64, _i64, _vp, _vp, _vp],
     "w4_linear_q4_0": [_vp, _i64, _vp, _i64, _i64, _vp, _vp, _i32, _vp],
     "w4_linear_backward_x_workspace_bytes": [_i64, _i64, _i64],
     "w4_linear_backward_x": [_vp, _i64, _vp, _vp, _i64, _i64, _vp, _i32, _vp, _sz, _vp],
@@ -267,6 +268,26 @@ def dequantize_q4_0(blocks: torch.Tensor, K: int, out_dtype=torch.float32,
     _check(_load().w4_dequantize_q4_0(_ptr(blocks), N, K, DTYPES[out.dtype], _ptr(out), _stream()),
            "w4_dequantize_q4_0")
     return out
+
+
+def q4_0_to_group32(blocks: torch.Tensor, K: int, out: tuple[torch.Tensor, torch.Tensor] | None = None):
+    """GGUF Q4_0 blocks (uint8 ``[N, K/32, 18]``) re-laid out once as the packed group-32 format:
+    returns ``(codes, scales)`` (uint8 ``[N, K/2]``, float32 ``[N, K/32]``; signed codes
+    ``c - 8``, scales ``d`` widened to fp32) for ``linear`` / ``Linear`` / ``dequantize``, which
+    then see exactly the blocks' dequantized weights."""
+    _need_cuda(blocks)
+    N = _q4_0_shape(blocks, K)
+    if out is None:
+        out = (torch.empty((N, K // 2), dtype=torch.uint8, device=blocks.device),
+               torch.empty((N, K // 32), dtype=torch.float32, device=blocks.device))
+    codes, scales = out
+    _need_cuda(codes, scales)
+    if not (codes.dtype == torch.uint8 and codes.is_contiguous() and codes.numel() == N * (K // 2)
+            and scales.dtype == torch.float32 and scales.is_contiguous() and scales.numel() == N * (K // 32)):
+        raise ValueError("out must be contiguous uint8 [N, K/2] codes and float32 [N, K/32] scales")
+    _check(_load().w4_q4_0_to_group32(_ptr(blocks), N, K, _ptr(codes), _ptr(scales), _stream()),
+           "w4_q4_0_to_group32")
+    return codes, scales
 
 
 def linear_q4_0(x: torch.Tensor, blocks: torch.Tensor, bias: torch.Tensor | None = None,

@@ -28,6 +28,9 @@
 //   * q4_0_linear_plain_kernel: any M and K (a multiple of 32), one warp per (row, 4 tokens),
 //     lanes striding over blocks, exact fp32 weights, fp32 accumulation: the floor.
 //   * q4_0_dequant_kernel: one thread per block, 32 outputs.
+//   * q4_0_to_group32_kernel: one thread per block, the block re-laid out as a group of the
+//     packed group-32 format (signed codes c - 8, the scale widened to fp32), once per weight:
+//     every group-32 entry point then reads the same dequantized weights.
 #include <cuda.h>
 
 #include <mutex>
@@ -318,6 +321,39 @@ __global__ void __launch_bounds__(256) q4_0_dequant_kernel(const uint8_t *__rest
   }
 }
 
+// One thread per block: the block's 16 code bytes become the 16 bytes of its 32-column group
+// in the packed group-32 layout (column 2b in the low nibble of byte b, column 2b + 1 in the
+// high one) holding the signed code c - 8 as a two's-complement nibble (c ^ 8), and the
+// binary16 scale its exact fp32 value. Block i of the weight is group i % (K/32) of row
+// i / (K/32), so its codes start at byte 16 i and its scale is scales[i].
+__global__ void __launch_bounds__(256) q4_0_to_group32_kernel(const uint8_t *__restrict__ blocks, int64_t nblocks,
+                                                              uint8_t *__restrict__ codes,
+                                                              float *__restrict__ scales, bool vec) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= nblocks) return;
+  const uint8_t *bp = blocks + i * kQBlockBytes;
+  uint32_t c[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) c[j] = bp[2 + j];
+  uint32_t out[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int b = 0; b < 16; ++b) {
+    // columns 2b, 2b + 1: elements below 16 are low nibbles of code bytes 2b, 2b + 1; the
+    // rest are high nibbles of bytes 2b - 16, 2b - 15
+    const uint32_t lo = b < 8 ? (c[2 * b] & 15u) : (c[2 * b - 16] >> 4);
+    const uint32_t hi = b < 8 ? (c[2 * b + 1] & 15u) : (c[2 * b - 15] >> 4);
+    out[b / 4] |= ((lo | (hi << 4)) ^ 0x88u) << (8 * (b % 4));
+  }
+  uint8_t *o = codes + i * 16;
+  if (vec) {
+    *reinterpret_cast<uint4 *>(o) = make_uint4(out[0], out[1], out[2], out[3]);
+  } else {
+#pragma unroll
+    for (int b = 0; b < 16; ++b) o[b] = static_cast<uint8_t>(out[b / 4] >> (8 * (b % 4)));
+  }
+  scales[i] = half_bits_to_float(static_cast<uint32_t>(bp[0]) | (static_cast<uint32_t>(bp[1]) << 8));
+}
+
 cudaError_t ensure_q4_0_smem() {
   static std::mutex mu;
   static bool done[64] = {};
@@ -417,6 +453,16 @@ cudaError_t launch_q4_0_dequantize(const uint8_t *blocks, int64_t N, int64_t K, 
     case W4_F64: q4_0_dequant_kernel<double><<<gi, 256, 0, stream>>>(blocks, nb, static_cast<double *>(out)); break;
     default: return cudaErrorInvalidValue;
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_q4_0_to_group32(const uint8_t *blocks, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                                   cudaStream_t stream) {
+  const int64_t nb = N * (K / 32);
+  const int64_t grid = (nb + 255) / 256;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const bool vec = reinterpret_cast<uintptr_t>(codes) % 16 == 0;
+  q4_0_to_group32_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(blocks, nb, codes, scales, vec);
   return cudaGetLastError();
 }
 

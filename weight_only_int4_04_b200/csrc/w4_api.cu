@@ -337,6 +337,16 @@ w4_status w4_dequantize_q4_0(const uint8_t *blocks, int64_t N, int64_t K, w4_dty
   return e == cudaSuccess ? W4_OK : cuda_fail(e);
 }
 
+w4_status w4_q4_0_to_group32(const uint8_t *blocks, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                             w4_stream_t stream) {
+  const NvtxRange nvtx_range("w4_q4_0_to_group32");
+  if (!blocks || !codes || !scales) return W4_ERR_NULL;
+  if (!sizes_ok(N, K) || K % 32 != 0) return W4_ERR_SHAPE;
+  const cudaError_t e =
+      w4i::launch_q4_0_to_group32(blocks, N, K, codes, scales, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? W4_OK : cuda_fail(e);
+}
+
 w4_status w4_linear_q4_0(const void *x, int64_t M, const uint8_t *blocks, int64_t N, int64_t K,
                          const float *bias, void *y, w4_dtype y_dtype, w4_stream_t stream) {
   const NvtxRange nvtx_range("w4_linear_q4_0");

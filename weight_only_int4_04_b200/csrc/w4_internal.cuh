@@ -81,6 +81,8 @@ cudaError_t launch_q4_0_linear(const __nv_bfloat16 *x, int64_t M, const uint8_t 
                                const float *bias, void *y, int y_dtype, bool prefetch, int32_t *err,
                                cudaStream_t stream);
 bool q4_0_gemv_supports(const void *x, int64_t M, const uint8_t *blocks, int64_t N, int64_t K, int y_dtype);
+cudaError_t launch_q4_0_to_group32(const uint8_t *blocks, int64_t N, int64_t K, uint8_t *codes, float *scales,
+                                   cudaStream_t stream);
 cudaError_t launch_q4_0_dequantize(const uint8_t *blocks, int64_t N, int64_t K, int out_dtype, void *out,
                                    cudaStream_t stream);
 
