@@ -52,6 +52,30 @@ def test_lora_merge_bit_exact(w4, NKr):
     assert torch.equal(dc, co) and torch.equal(ds, so)
 
 
+@pytest.mark.parametrize("NKr", [(2050, 4100, 16), (1024, 2048, 40), (4096, 4096, 0)])
+def test_lora_merge_row_tile_walk(w4, NKr):
+    # more 32-row tiles than a column tile's walkers: each CTA merges several row tiles in
+    # turn (next tile's codes fetched ahead, the rank slices re-staged per chunk when r > 32)
+    N, K, r = NKr
+    codes, s, b, a = lora_case(N, K, r, 3 * N + K + r)
+    c = 2.0 / max(r, 1)
+    q2, s2 = O.lora_merge(codes, s, K, b, a, c)
+    co, so = w4.lora_merge(dev(codes), dev(s), K, dev(b) if r else None, dev(a) if r else None, c)
+    assert np.array_equal(co.cpu().numpy(), O.pack_nibbles(q2)), NKr
+    assert np.array_equal(so.cpu().numpy().view(np.uint32), s2.view(np.uint32)), NKr
+
+
+def test_lora_merge_full_size_in_place(w4):
+    # the merge the bench times: rank 16 into (14336, 4096), in place, every code and scale
+    N, K, r = 14336, 4096, 16
+    codes, s, b, a = lora_case(N, K, r, 99)
+    q2, s2 = O.lora_merge(codes, s, K, b, a, 2.0 / r)
+    dc, ds = dev(codes), dev(s)
+    w4.lora_merge(dc, ds, K, dev(b), dev(a), 2.0 / r, out=(dc, ds))
+    assert np.array_equal(dc.cpu().numpy(), O.pack_nibbles(q2))
+    assert np.array_equal(ds.cpu().numpy().view(np.uint32), s2.view(np.uint32))
+
+
 def test_lora_merge_ties_and_near_ties(w4):
     # merged values on and 2^-22 beside half-integers of the new scale, with scales whose
     # reciprocal is exact in fp32 (1, 2^-20) and inexact (3, 3/8, 1/3, 5, 7): the codes round
