@@ -36,8 +36,29 @@ int grid_for(int64_t work_items, int items_per_block) {
 // RTN quantize + pack (page "loopq/packed_weight.py", pack_weight; rounding and clip of
 // page "gemma/peft/_quantization_utils.py", uniform_quantize).
 // Eight lanes cooperate on one group of 32 columns, four columns per lane, so one warp
-// instruction reads four consecutive groups (512 contiguous bytes of W).
+// instruction reads four consecutive groups (512 contiguous bytes of W). A lane's (row,
+// group) advances by a fixed step per trip of the grid-stride loop (no division inside it).
+//
+// The code is rne(fl32(w / s)) clamped to [-7, 7], s = max(fl32(amax / 7), 2^-126), formed
+// without a division per element: |w / s| <= 7 / (1 - 2^-24) because |w| <= amax and
+// s >= amax / 7 rounded down by at most half an ulp (or s = 2^-126 > amax / 7), so the clamp
+// never acts. With y = fl32(1 / s), x = fl32(w * y) is within 2^-20 of w / s and fl32(w / s)
+// within 2^-22 of it (|w / s| < 8), so both round to the same integer unless x is within
+// 2^-19 of a half-integer; a lane whose four values come within 2^-18 of one takes the IEEE
+// quotients instead. Adding 1.5 * 2^23 rounds to an integer, half to even, and leaves its
+// two's-complement nibble in the low bits.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t rtn_nibble(float w, float y, bool &near) {
+  const float x = __fmul_rn(w, y);
+  const float xm = __fadd_rn(x, 12582912.0f);
+  near |= fabsf(__fsub_rn(x, __fsub_rn(xm, 12582912.0f))) > 0.5f - 0x1p-18f;
+  return __float_as_uint(xm) & 15u;
+}
+
+__device__ __forceinline__ uint32_t rtn_nibble_exact(float w, float s) {
+  return __float_as_uint(__fadd_rn(__fdiv_rn(w, s), 12582912.0f)) & 15u;
+}
+
 __global__ void __launch_bounds__(kThreads) quantize_rtn_kernel(const float *__restrict__ W,
                                                                 int64_t N, int64_t K,
                                                                 uint8_t *__restrict__ codes,
@@ -50,16 +71,19 @@ __global__ void __launch_bounds__(kThreads) quantize_rtn_kernel(const float *__r
   const int sub = lane & 7;
   const int64_t tasks = N * G;
   const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t warp_stride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t step = ((static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) * 4;  // tasks per trip
+  const int64_t dn = step / G, dg = step % G;
+  // this lane's task t = n * G + g (past the end on the last trips: then unused)
+  int64_t t = warp_id * 4 + (lane >> 3);
+  int64_t n = t / G, g = t % G;
   bool bad = false;
   // A warp owns four consecutive tasks per trip; the trip count is warp-uniform so every
   // lane reaches the shuffles below (lanes past the end work on zeros and store nothing).
-  for (int64_t wb = warp_id * 4; wb < tasks; wb += warp_stride * 4) {
-    const int64_t t = wb + (lane >> 3);
+  for (int64_t wb = warp_id * 4; wb < tasks; wb += step) {
     const bool active = t < tasks;
-    const int64_t n = active ? t / G : 0, g = active ? t % G : 0;
-    const int64_t c0 = 32 * g + 4 * sub;
-    const float *row = W + n * K;
+    const int64_t na = active ? n : 0, ga = active ? g : 0;
+    const int64_t c0 = 32 * ga + 4 * sub;
+    const float *row = W + na * K;
     float w[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     if (!active) {
     } else if (vec_ok && c0 + 3 < K) {
@@ -80,21 +104,33 @@ __global__ void __launch_bounds__(kThreads) quantize_rtn_kernel(const float *__r
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
     // s = max(fl32(amax / 7), FLT_MIN): IEEE round-to-nearest divide.
     const float s = fmaxf(__fdiv_rn(amax, 7.0f), FLT_MIN);
+    const float y = __frcp_rn(s);
+    bool near = false;
     uint32_t nib[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      int q = __float2int_rn(__fdiv_rn(w[i], s));  // round half to even
-      q = q < -7 ? -7 : (q > 7 ? 7 : q);
-      nib[i] = (c0 + i < K) ? (static_cast<uint32_t>(q) & 15u) : 0u;  // pad nibble = 0
+    for (int i = 0; i < 4; ++i) nib[i] = rtn_nibble(w[i], y, near);
+    if (near) {  // rare: a value close to a half-integer takes the exact quotient
+#pragma unroll
+      for (int i = 0; i < 4; ++i) nib[i] = rtn_nibble_exact(w[i], s);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) nib[i] = (c0 + i < K) ? nib[i] : 0u;  // pad nibble = 0
     const uint8_t b0 = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
     const uint8_t b1 = static_cast<uint8_t>(nib[2] | (nib[3] << 4));
+    // advance this lane's task by one trip: t + step = (n + dn) G + (g + dg), one carry at most
+    t += step;
+    n += dn;
+    g += dg;
+    if (g >= G) {
+      g -= G;
+      ++n;
+    }
     if (!active) continue;
-    uint8_t *crow = codes + n * P;
+    uint8_t *crow = codes + na * P;
     const int64_t j = c0 / 2;
     if (j < P) crow[j] = b0;
     if (j + 1 < P) crow[j + 1] = b1;
-    if (sub == 0) scales[n * G + g] = s;
+    if (sub == 0) scales[na * G + ga] = s;
   }
   if (bad) *status = W4_ERR_NONFINITE;
 }
