@@ -42,17 +42,31 @@ int grid_for(int64_t work_items, int items_per_block) {
 // The code is rne(fl32(w / s)) clamped to [-7, 7], s = max(fl32(amax / 7), 2^-126), formed
 // without a division per element: |w / s| <= 7 / (1 - 2^-24) because |w| <= amax and
 // s >= amax / 7 rounded down by at most half an ulp (or s = 2^-126 > amax / 7), so the clamp
-// never acts. With y = fl32(1 / s), x = fl32(w * y) is within 2^-20 of w / s and fl32(w / s)
-// within 2^-22 of it (|w / s| < 8), so both round to the same integer unless x is within
-// 2^-19 of a half-integer; a lane whose four values come within 2^-18 of one takes the IEEE
-// quotients instead. Adding 1.5 * 2^23 rounds to an integer, half to even, and leaves its
-// two's-complement nibble in the low bits.
+// never acts. y = rcp.approx(s) is within one ulp of 1 / s (the PTX ISA's bound for
+// rcp.approx.f32; s and 1 / s are normal), so x = fl32(w * y) is within 1.51 * 2^-21 of
+// w / s and fl32(w / s) within 2^-22 of it (|w / s| < 8): both round to the same integer
+// unless x is within 2^-20 of a half-integer; a lane whose four values come within 2^-18 of
+// one takes the IEEE quotients instead. Adding 1.5 * 2^23 rounds to an integer, half to even,
+// and leaves its two's-complement nibble in the low bits.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t rtn_nibble(float w, float y, bool &near) {
   const float x = __fmul_rn(w, y);
   const float xm = __fadd_rn(x, 12582912.0f);
   near |= fabsf(__fsub_rn(x, __fsub_rn(xm, 12582912.0f))) > 0.5f - 0x1p-18f;
   return __float_as_uint(xm) & 15u;
+}
+
+__device__ __forceinline__ float rcp_approx(float s) {
+  float y;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(y) : "f"(s));
+  return y;
+}
+
+// max that returns NaN when either input is NaN, so one test of the amax covers the values
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t rtn_nibble_exact(float w, float s) {
@@ -95,16 +109,14 @@ __global__ void __launch_bounds__(kThreads) quantize_rtn_kernel(const float *__r
     }
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      bad |= !isfinite(w[i]);
-      amax = fmaxf(amax, fabsf(w[i]));
-    }
+    for (int i = 0; i < 4; ++i) amax = max_nan(amax, fabsf(w[i]));
+    bad |= !(amax <= FLT_MAX);  // a NaN or an infinity among this lane's values
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
     // s = max(fl32(amax / 7), FLT_MIN): IEEE round-to-nearest divide.
     const float s = fmaxf(__fdiv_rn(amax, 7.0f), FLT_MIN);
-    const float y = __frcp_rn(s);
+    const float y = rcp_approx(s);
     bool near = false;
     uint32_t nib[4];
 #pragma unroll
@@ -113,10 +125,12 @@ __global__ void __launch_bounds__(kThreads) quantize_rtn_kernel(const float *__r
 #pragma unroll
       for (int i = 0; i < 4; ++i) nib[i] = rtn_nibble_exact(w[i], s);
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) nib[i] = (c0 + i < K) ? nib[i] : 0u;  // pad nibble = 0
-    const uint8_t b0 = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
-    const uint8_t b1 = static_cast<uint8_t>(nib[2] | (nib[3] << 4));
+    // columns past K: pad nibble 0
+    const int64_t left = K - c0;
+    const uint32_t colmask = left >= 4 ? 0xFFFFu : (left <= 0 ? 0u : (1u << (4 * left)) - 1u);
+    const uint32_t w16 = (nib[0] | (nib[1] << 4) | (nib[2] << 8) | (nib[3] << 12)) & colmask;
+    const uint8_t b0 = static_cast<uint8_t>(w16);
+    const uint8_t b1 = static_cast<uint8_t>(w16 >> 8);
     // advance this lane's task by one trip: t + step = (n + dn) G + (g + dg), one carry at most
     t += step;
     n += dn;
